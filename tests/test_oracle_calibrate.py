@@ -1,0 +1,142 @@
+"""Pins of the oracle's offline calibration (basis U, coefficient map R).
+
+The pages fix only that queries are approximated on a low-rank basis fixed
+offline, weighted by the state.  The pins check the algebra any such
+least-squares map must satisfy, and check by brute force on tiny heads -- a
+direct minimisation over the calibration data, not through the Gram formula --
+that the oracle's basis minimises the averaged squared read error.
+"""
+
+import numpy as np
+import pytest
+from scipy import optimize
+
+from oracle import calibration as cal
+
+
+def _data(rng, Ns, Nq, dk, dv, rank=None, noise=0.1):
+    S = rng.standard_normal((Ns, dk, dv)) * rng.uniform(0.2, 2.0, (1, dk, 1))
+    if rank is None:
+        q = rng.standard_normal((Nq, dk)) * rng.uniform(0.3, 1.5, (1, dk))
+    else:
+        Q0 = np.linalg.qr(rng.standard_normal((dk, rank)))[0]
+        q = rng.standard_normal((Nq, rank)) @ Q0.T + noise * rng.standard_normal((Nq, dk))
+    return S, q
+
+
+def _ridged_gram(S, ridge=1e-8):
+    G = cal.gram_states(S)
+    return G + ridge * np.trace(G) / G.shape[0] * np.eye(G.shape[0])
+
+
+@pytest.mark.parametrize("r", [1, 3, 8])
+def test_algebraic_properties(r):
+    rng = np.random.default_rng(21)
+    dk, dv = 16, 12
+    S, q = _data(rng, 40, 300, dk, dv)
+    U, R = cal.calibrate(S, q, r)
+    G = _ridged_gram(S)
+    Pi = U @ R
+    np.testing.assert_allclose(R @ U, np.eye(r), atol=1e-10)
+    np.testing.assert_allclose(Pi @ Pi, Pi, atol=1e-10)
+    np.testing.assert_allclose(G @ Pi, (G @ Pi).T, atol=1e-9 * np.abs(G).max())
+    np.testing.assert_allclose(U.T @ G @ (np.eye(dk) - Pi), 0.0, atol=1e-9 * np.abs(G).max())
+
+
+def _data_objective(S, q, U):
+    """Mean over states and queries of ||S^T q - S^T U c||^2 with c the per-query
+    least-squares coefficients, solved on the stacked data (all states at once)."""
+    A = np.concatenate([s.T @ U for s in S], axis=0)  # (Ns*dv, r)
+    Y = np.concatenate([np.einsum("ic,ni->cn", s, q) for s in S], axis=0)  # (Ns*dv, Nq)
+    c, *_ = np.linalg.lstsq(A, Y, rcond=None)
+    res = Y - A @ c
+    return float(np.sum(res ** 2) / (S.shape[0] * q.shape[0]))
+
+
+def _sphere(n):
+    i = np.arange(n) + 0.5
+    phi = np.arccos(1 - i / n)  # upper hemisphere: u and -u span the same line
+    th = np.pi * (1 + 5 ** 0.5) * i
+    return np.stack([np.cos(th) * np.sin(phi), np.sin(th) * np.sin(phi), np.cos(phi)], 1)
+
+
+def _proj(U, R):
+    return U @ R
+
+
+def test_brute_force_rank1_dk3():
+    rng = np.random.default_rng(22)
+    S, q = _data(rng, 6, 60, 3, 4)
+    U, R = cal.calibrate(S, q, 1, ridge=0.0)
+    grid = _sphere(4000)
+    vals = np.array([_data_objective(S, q, u[:, None]) for u in grid])
+    u0 = grid[np.argmin(vals)]
+    f = lambda x: _data_objective(S, q, (x / np.linalg.norm(x))[:, None])  # noqa
+    x = optimize.minimize(f, u0, method="Nelder-Mead",
+                          options={"xatol": 1e-12, "fatol": 1e-15, "maxiter": 20000}).x
+    best = x / np.linalg.norm(x)
+    ours = U[:, 0] / np.linalg.norm(U[:, 0])
+    assert _data_objective(S, q, U) <= f(best) * (1 + 1e-9)
+    assert min(np.linalg.norm(best - ours), np.linalg.norm(best + ours)) < 1e-4
+
+
+def test_brute_force_rank2_dk3():
+    rng = np.random.default_rng(23)
+    S, q = _data(rng, 5, 80, 3, 3)
+    U, R = cal.calibrate(S, q, 2, ridge=0.0)
+
+    def basis(n):
+        n = n / np.linalg.norm(n)
+        return np.linalg.svd(np.eye(3) - np.outer(n, n))[0][:, :2]
+
+    grid = _sphere(4000)
+    vals = np.array([_data_objective(S, q, basis(n)) for n in grid])
+    f = lambda x: _data_objective(S, q, basis(x))  # noqa
+    x = optimize.minimize(f, grid[np.argmin(vals)], method="Nelder-Mead",
+                          options={"xatol": 1e-12, "fatol": 1e-15, "maxiter": 20000}).x
+    Ub = basis(x)
+    assert _data_objective(S, q, U) <= f(x) * (1 + 1e-9)
+    # same span: the G-weighted projector of the brute-force basis equals the oracle's
+    G = cal.gram_states(S)
+    Rb = np.linalg.solve(Ub.T @ G @ Ub, Ub.T @ G)
+    np.testing.assert_allclose(Ub @ Rb, U @ R, atol=1e-4)
+
+
+def test_isotropic_state_weight_is_query_pca():
+    """With G a multiple of I the basis spans the top principal directions of the queries."""
+    rng = np.random.default_rng(24)
+    dk, r = 12, 4
+    O = np.linalg.qr(rng.standard_normal((dk, dk)))[0]
+    S = np.stack([O * 1.7, -O * 1.7])  # S S^T = 1.7^2 I for both states
+    q = rng.standard_normal((500, dk)) * np.linspace(3.0, 0.2, dk)[None, :]
+    U, R = cal.calibrate(S, q, r, ridge=0.0)
+    Vt = np.linalg.svd(q, full_matrices=False)[2]
+    Ppca = Vt[:r].T @ Vt[:r]
+    np.testing.assert_allclose(U @ R, Ppca, atol=1e-9)
+
+
+def test_exact_low_rank_queries_are_reproduced():
+    rng = np.random.default_rng(25)
+    dk, dv, r = 16, 8, 5
+    S, q = _data(rng, 30, 200, dk, dv, rank=r, noise=0.0)
+    U, R = cal.calibrate(S, q, r)
+    np.testing.assert_allclose(q @ (U @ R).T, q, atol=1e-9)
+
+
+def test_complete_rank_is_identity():
+    rng = np.random.default_rng(26)
+    S, q = _data(rng, 20, 100, 8, 8)
+    U, R = cal.calibrate(S, q, 8)
+    np.testing.assert_allclose(U @ R, np.eye(8), atol=1e-9)
+
+
+def test_beats_query_pca_and_random_bases():
+    rng = np.random.default_rng(27)
+    dk, dv, r = 16, 16, 4
+    S, q = _data(rng, 50, 400, dk, dv, rank=8, noise=0.2)
+    U, R = cal.calibrate(S, q, r, ridge=0.0)
+    ours = _data_objective(S, q, U)
+    Vt = np.linalg.svd(q, full_matrices=False)[2]
+    assert ours <= _data_objective(S, q, Vt[:r].T) * (1 + 1e-12)
+    for _ in range(20):
+        assert ours <= _data_objective(S, q, rng.standard_normal((dk, r))) * (1 + 1e-12)

@@ -114,8 +114,9 @@ int orc_num_threads(void)
 
 /* Per-step exact recurrence over T tokens for N heads (the full-read path):
  * for t = 0..T-1: S <- token t; if Q: O[t] = S^T Q[t].  With bf16_state the
- * state is rounded to bf16 after every token, as a path that stores S in bf16
- * and writes it back every step.
+ * state is rounded to bf16 after every token (after that token's read, which
+ * sees the unrounded update), as a path that stores S in bf16 and writes it
+ * back every step.
  *   S [N][dk][dv] in/out;  K [T][N][dk];  V [T][N][dv];  A [T][N][na]
  *   (na = dk for KDA, else 1);  Bt [T][N] (ignored for Mamba-2, may be NULL);
  *   Q [T][N][dk] or NULL;  O [T][N][dv] or NULL. */
@@ -133,9 +134,9 @@ int orc_exact_steps(int kind, int N, int dk, int dv, int T, double *S, const dou
             size_t tn = (size_t)t * N + n;
             double beta = kind == ORC_MAMBA2 ? 1.0 : Bt[tn];
             token_update(kind, dk, dv, Sn, K + tn * dk, V + tn * dv, A + tn * na, beta);
+            if (Q && O) read_state(dk, dv, Sn, Q + tn * dk, O + tn * dv);
             if (bf16_state)
                 for (int e = 0; e < dk * dv; ++e) Sn[e] = to_bf16(Sn[e]);
-            if (Q && O) read_state(dk, dv, Sn, Q + tn * dk, O + tn * dv);
         }
     }
     return 0;

@@ -1,0 +1,186 @@
+/*
+ * sketchssm.h -- C ABI of the SketchSSM windowed linear-attention decode for
+ * NVIDIA B200 (sm_100a).
+ *
+ * Method: "SketchSSM: Write to the Full State, Read from a Compact Sketch"
+ * (arXiv 2609.33051v1), Abstract; agihunt digest of the same paper, bullets
+ * "Core idea", "Mechanism details" and "Error control".  Keys and values are
+ * buffered for a window of W decode steps (the ReplaySSM buffering the abstract
+ * builds on).  Once per window one kernel reads each head's full recurrent
+ * state S, applies the buffered tokens exactly and, in the same pass, refreshes
+ * a compact sketch P = S^T U against an offline basis U.  Each decode step in
+ * the window reads only the sketch: it carries its query back to the
+ * window-start state through the buffered tokens (q~), adds the exact
+ * contribution of those tokens, and reconstructs the state part as P (R q~).
+ * Approximation error never enters S.
+ *
+ * Recurrences (per head; S is dk x dv, i a key channel, c a value channel):
+ *   SKSSM_MAMBA2  S <- a S + k v^T                     a scalar per token/head
+ *   SKSSM_GDN     S <- a (I - b k k^T) S + b k v^T     a, b scalars
+ *   SKSSM_KDA     S <- (I - b k k^T) diag(a) S + b k v^T   a per key channel
+ * Read: o = S^T q after the step's own token has been applied.
+ *
+ * ---------------------------------------------------------------------------
+ * Conventions shared by every entry point
+ *   - Every array pointer is DEVICE memory owned by the caller, on the device
+ *     that is current for the calling thread, densely packed (C order), and
+ *     16-byte aligned unless stated otherwise.  The library keeps no pointer
+ *     after a call returns and allocates no memory.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
+ *     asynchronous on it; kernel-side faults surface at the caller's next
+ *     synchronisation.
+ *   - Every call validates its arguments on the host before launching anything
+ *     and returns SKSSM_OK (0) or a negative sketchssm_status; on error nothing
+ *     was launched and no memory was touched.
+ *   - Storage layouts (N = B*H heads, flat head index n = b*H + h):
+ *       S      [B][H][dv][dk]  state, stored transposed: row c holds column c of
+ *                              S, i.e. S_T[n][c][i] = S[i][c]; dtype state_dtype
+ *       P      [B][H][dv][r]   fp32 sketch, P[n][c][m] = sum_i S[i][c] U[i][m]
+ *       U      [H][dk][r]      fp32 basis (per head h, shared by all b)
+ *       R      [H][r][dk]      fp32 coefficient map, c = R q~
+ *       window buffer, time-major, slot t = token t of the window:
+ *       k      [W][B][H][dk]   qkv_dtype
+ *       v      [W][B][H][dv]   qkv_dtype
+ *       alpha  [W][B][H]       fp32 decay (SKSSM_KDA: [W][B][H][dk]); 4-byte aligned
+ *       beta   [W][B][H]       fp32 (ignored, may be NULL, for SKSSM_MAMBA2); 4-byte aligned
+ *       q      [B][H][dk]      qkv_dtype, the current step's query
+ *       o      [B][H][dv]      fp32 output
+ *   - Supported sizes: dk in {64, 128}; dv in {64, 128}; 1 <= r <= 32 or r == dk;
+ *     1 <= W <= 64; B >= 1, H >= 1, B*H < 2^31.  Other sizes: SKSSM_ERR_DIMS.
+ * ---------------------------------------------------------------------------
+ */
+#ifndef SKETCHSSM_H
+#define SKETCHSSM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { SKSSM_MAMBA2 = 0, SKSSM_GDN = 1, SKSSM_KDA = 2 } sketchssm_kind;
+typedef enum { SKSSM_F32 = 0, SKSSM_BF16 = 1 } sketchssm_dtype;
+
+typedef enum {
+    SKSSM_OK = 0,
+    SKSSM_ERR_NULL = -1,      /* a required pointer is NULL */
+    SKSSM_ERR_DIMS = -2,      /* unsupported kind / sizes */
+    SKSSM_ERR_RANGE = -3,     /* j, n_tokens, Nq or Ns out of range */
+    SKSSM_ERR_ALIGN = -4,     /* a pointer breaks its alignment rule */
+    SKSSM_ERR_DTYPE = -5,     /* unsupported storage dtype */
+    SKSSM_ERR_CUDA = -6,      /* a CUDA runtime call or launch failed */
+    SKSSM_ERR_WORKSPACE = -7  /* workspace missing or too small */
+} sketchssm_status;
+
+typedef struct sketchssm_dims {
+    int32_t kind;        /* sketchssm_kind */
+    int32_t B, H;        /* sequences in the batch, heads per sequence */
+    int32_t dk, dv;      /* key (state rows) and value (state columns) widths */
+    int32_t r;           /* sketch rank */
+    int32_t W;           /* window length: slots in the token buffer */
+    int32_t state_dtype; /* storage of S: SKSSM_F32 or SKSSM_BF16 */
+    int32_t qkv_dtype;   /* storage of q, k, v: SKSSM_F32 or SKSSM_BF16 */
+} sketchssm_dims;
+
+/* Human-readable text of a status code (static string, never NULL). */
+const char *sketchssm_status_string(int status);
+
+/* ABI version of this library: major * 10000 + minor * 100 + patch. */
+int sketchssm_version(void);
+
+/*
+ * sketchssm_update_window -- the once-per-window state update and sketch refresh.
+ * Defines: SketchSSM abstract (one full-state read per state update precomputes
+ * the basis outputs into the sketch); digest bullet "Error control" (the same
+ * kernel updates the full state and refreshes the sketch).
+ * For every head: apply buffered tokens t = 0 .. n_tokens-1 of the window
+ * buffer to S, in order, exactly (fp32 arithmetic); store S (rounded to
+ * state_dtype, nearest-even, for SKSSM_BF16); then write P = S_stored^T U.
+ * n_tokens = 0 is a sketch refresh only (S is read, not written).
+ *   S        in/out [B][H][dv][dk] state_dtype
+ *   P        out    [B][H][dv][r] fp32
+ *   U        in     [H][dk][r] fp32
+ *   k, v, alpha, beta  in: window buffer slots 0..n_tokens-1 (NULL allowed when
+ *            n_tokens == 0; beta NULL allowed for SKSSM_MAMBA2)
+ * Errors: ERR_NULL, ERR_DIMS, ERR_DTYPE, ERR_RANGE (n_tokens < 0 or > W),
+ * ERR_ALIGN, ERR_CUDA.
+ */
+int sketchssm_update_window(const sketchssm_dims *dims, void *S, float *P, const float *U,
+                            const void *k, const void *v, const float *alpha, const float *beta,
+                            int n_tokens, void *stream);
+
+/*
+ * sketchssm_decode_step -- one decode step inside a window, reading only the sketch.
+ * Defines: SketchSSM abstract (each decode step combines the sketch vectors with
+ * query-dependent coefficients instead of reading the full state); digest
+ * bullet "Mechanism details" (a query that is a combination of basis vectors
+ * has as output the same combination of the stored outputs).
+ * Step j of the window: tokens 0..j-1 of the buffer are not yet in the state
+ * whose sketch is P (token j-1 is this step's own token).  Per head:
+ *     w <- q;  o_buf <- 0
+ *     for t = j-1 down to 0:  x = k_t . w;  s = b_t x (b = 1 for Mamba-2);
+ *                             o_buf += s v_t;  w <- M_t^T w
+ *         (M_t^T w: Mamba-2 a_t w; GDN a_t (w - s k_t); KDA a_t (.) (w - s k_t))
+ *     o = P (R w) + o_buf
+ *   P in [B][H][dv][r];  R in [H][r][dk];  q in [B][H][dk];
+ *   k, v, alpha, beta in: window buffer slots 0..j-1;  o out [B][H][dv] fp32.
+ * Errors: ERR_NULL, ERR_DIMS, ERR_DTYPE, ERR_RANGE (j < 1 or j > W), ERR_ALIGN,
+ * ERR_CUDA.
+ */
+int sketchssm_decode_step(const sketchssm_dims *dims, const float *P, const float *R,
+                          const void *q, const void *k, const void *v, const float *alpha,
+                          const float *beta, int j, float *o, void *stream);
+
+/*
+ * sketchssm_fullread_decode -- the baseline: one decode step with a full-state
+ * read, as a standard serving engine does it (SketchSSM abstract, "standard
+ * vLLM baseline"; digest bullet "Background": the full recurrent state is read
+ * at every decode step).  Per head: S <- M S + b k v^T with this step's token,
+ * S stored back (state_dtype), o = S^T q from the updated fp32 values.
+ *   S in/out [B][H][dv][dk];  q, k in [B][H][dk];  v in [B][H][dv];
+ *   alpha in [B][H] (KDA [B][H][dk]);  beta in [B][H] (NULL for Mamba-2);
+ *   o out [B][H][dv] fp32.  (One window slot is a valid token argument.)
+ * Errors: ERR_NULL, ERR_DIMS, ERR_DTYPE, ERR_ALIGN, ERR_CUDA.
+ */
+int sketchssm_fullread_decode(const sketchssm_dims *dims, void *S, const void *q, const void *k,
+                              const void *v, const float *alpha, const float *beta, float *o,
+                              void *stream);
+
+/*
+ * sketchssm_calibrate_workspace_bytes -- device workspace that
+ * sketchssm_calibrate_basis needs for these sizes (0 if dims are invalid).
+ */
+size_t sketchssm_calibrate_workspace_bytes(const sketchssm_dims *dims, int Nq, int Ns);
+
+/*
+ * sketchssm_calibrate_basis -- offline basis U and coefficient map R, per head.
+ * Defines: SketchSSM abstract (low-rank, state-weighted query approximation on
+ * basis vectors fixed offline); digest bullet "Core idea".  With
+ *     G = (1/Ns) sum_s S_s S_s^T + ridge (tr G / dk) I     (state weighting)
+ *     C = (1/Nq) sum_n q_n q_n^T                           (query second moment)
+ * the basis spans the r-dimensional subspace that minimises the calibration-
+ * averaged squared read error E ||S^T (q - U R q)||^2, and R = (U^T G U)^-1 U^T G
+ * is the state-weighted least-squares coefficient map.  Computed in fp64
+ * (Cholesky G = L L^T, Jacobi eigenvectors V_r of L^T C L with the r largest
+ * eigenvalues, U = L^-T V_r, R = V_r^T L^T, so that R U = I); stored fp32.
+ *   q_cal  in  [H][Nq][dk] fp32 calibration queries, Nq >= 1
+ *   S_cal  in  [Ns][H][dv][dk] calibration states in the S layout, state_dtype,
+ *              Ns >= 1 (the B field of dims is ignored here)
+ *   ridge  >= 0, relative diagonal guard (1e-8 is a good default)
+ *   U out [H][dk][r] fp32;  R out [H][r][dk] fp32
+ *   workspace: device scratch of at least
+ *              sketchssm_calibrate_workspace_bytes(dims, Nq, Ns) bytes, 256-byte
+ *              aligned, owned by the caller; contents on entry are ignored.
+ * Offline: not on the decode path.  Errors: ERR_NULL, ERR_DIMS, ERR_DTYPE,
+ * ERR_RANGE, ERR_ALIGN, ERR_WORKSPACE, ERR_CUDA.
+ */
+int sketchssm_calibrate_basis(const sketchssm_dims *dims, const float *q_cal, int Nq,
+                              const void *S_cal, int Ns, double ridge, float *U, float *R,
+                              void *workspace, size_t workspace_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SKETCHSSM_H */

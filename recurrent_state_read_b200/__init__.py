@@ -1,0 +1,183 @@
+"""Python binding of the SketchSSM windowed-decode library (libsketchssm.so, sm_100a).
+
+Argument marshalling only: every function below checks that it was handed
+device tensors of the right dtype and size, then calls the C entry point of
+the same name (include/sketchssm.h) with raw pointers and the current torch
+CUDA stream.  All arithmetic runs in the library's CUDA kernels; there is no
+CPU fallback, and calling any entry point without the built library raises.
+
+Layouts (N = B*H heads, see include/sketchssm.h):
+    S [B,H,dv,dk]  (state, transposed storage)   P [B,H,dv,r] fp32
+    U [H,dk,r] fp32      R [H,r,dk] fp32
+    window buffer: k [W,B,H,dk], v [W,B,H,dv], alpha [W,B,H] (KDA [W,B,H,dk]), beta [W,B,H]
+    q [B,H,dk], o [B,H,dv] fp32
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsketchssm.so")
+
+KIND = {"mamba2": 0, "gdn": 1, "kda": 2}
+DTYPE = {torch.float32: 0, torch.bfloat16: 1}
+EXPORTS = (
+    "sketchssm_status_string",
+    "sketchssm_version",
+    "sketchssm_update_window",
+    "sketchssm_decode_step",
+    "sketchssm_fullread_decode",
+    "sketchssm_calibrate_workspace_bytes",
+    "sketchssm_calibrate_basis",
+)
+
+
+class sketchssm_dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("kind", "B", "H", "dk", "dv", "r", "W", "state_dtype", "qkv_dtype")]
+
+    def __repr__(self):
+        return "sketchssm_dims(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+class SketchSSMError(RuntimeError):
+    def __init__(self, fn: str, status: int, text: str):
+        super().__init__(f"{fn} failed: status {status} ({text})")
+        self.status = status
+
+
+_lib = None
+
+
+def library() -> ctypes.CDLL:
+    """The loaded CUDA library.  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m recurrent_state_read_b200.build` (nvcc, sm_100a)")
+        lib = ctypes.CDLL(LIB_PATH)
+        P = ctypes.c_void_p
+        D = ctypes.POINTER(sketchssm_dims)
+        i = ctypes.c_int
+        lib.sketchssm_status_string.argtypes = [i]
+        lib.sketchssm_status_string.restype = ctypes.c_char_p
+        lib.sketchssm_version.argtypes = []
+        lib.sketchssm_version.restype = i
+        lib.sketchssm_update_window.argtypes = [D, P, P, P, P, P, P, P, i, P]
+        lib.sketchssm_decode_step.argtypes = [D, P, P, P, P, P, P, P, i, P, P]
+        lib.sketchssm_fullread_decode.argtypes = [D, P, P, P, P, P, P, P, P]
+        lib.sketchssm_calibrate_workspace_bytes.argtypes = [D, i, i]
+        lib.sketchssm_calibrate_workspace_bytes.restype = ctypes.c_size_t
+        lib.sketchssm_calibrate_basis.argtypes = [D, P, i, P, i, ctypes.c_double, P, P, P,
+                                                  ctypes.c_size_t, P]
+        for f in ("sketchssm_update_window", "sketchssm_decode_step", "sketchssm_fullread_decode",
+                  "sketchssm_calibrate_basis"):
+            getattr(lib, f).restype = i
+        _lib = lib
+    return _lib
+
+
+def dims(kind, B, H, dk, dv, r, W, state_dtype=torch.float32, qkv_dtype=torch.bfloat16) -> sketchssm_dims:
+    k = KIND[kind] if isinstance(kind, str) else int(kind)
+    return sketchssm_dims(k, B, H, dk, dv, r, W, DTYPE[state_dtype], DTYPE[qkv_dtype])
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor], name: str, numel: int = None, dtype=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name}: expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if numel is not None and t.numel() < numel:
+        raise ValueError(f"{name}: needs at least {numel} elements, has {t.numel()}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dt(code: int):
+    return torch.float32 if code == 0 else torch.bfloat16
+
+
+def _check(fn: str, rc: int):
+    if rc != 0:
+        raise SketchSSMError(fn, rc, library().sketchssm_status_string(rc).decode())
+
+
+def _token_ptrs(d: sketchssm_dims, n: int, k, v, alpha, beta):
+    NH = d.B * d.H
+    qt = _dt(d.qkv_dtype)
+    na = d.dk if d.kind == KIND["kda"] else 1
+    return (_ptr(k, "k", n * NH * d.dk, qt), _ptr(v, "v", n * NH * d.dv, qt),
+            _ptr(alpha, "alpha", n * NH * na, torch.float32),
+            _ptr(beta, "beta", n * NH, torch.float32))
+
+
+def sketchssm_update_window(d: sketchssm_dims, S, P, U, k, v, alpha, beta, n_tokens: int, stream=None):
+    """Apply window-buffer tokens 0..n_tokens-1 to S exactly and refresh P = S^T U (one kernel)."""
+    NH = d.B * d.H
+    args = (_ptr(S, "S", NH * d.dv * d.dk, _dt(d.state_dtype)), _ptr(P, "P", NH * d.dv * d.r, torch.float32),
+            _ptr(U, "U", d.H * d.dk * d.r, torch.float32))
+    toks = _token_ptrs(d, n_tokens, k, v, alpha, beta) if n_tokens > 0 else (None,) * 4
+    _check("sketchssm_update_window",
+           library().sketchssm_update_window(ctypes.byref(d), *args, *toks, int(n_tokens),
+                                             ctypes.c_void_p(_stream(stream))))
+
+
+def sketchssm_decode_step(d: sketchssm_dims, P, R, q, k, v, alpha, beta, j: int, o, stream=None):
+    """Decode step j of the window from the sketch P and window-buffer tokens 0..j-1 into o."""
+    NH = d.B * d.H
+    toks = _token_ptrs(d, j, k, v, alpha, beta)
+    _check("sketchssm_decode_step", library().sketchssm_decode_step(
+        ctypes.byref(d), _ptr(P, "P", NH * d.dv * d.r, torch.float32),
+        _ptr(R, "R", d.H * d.r * d.dk, torch.float32), _ptr(q, "q", NH * d.dk, _dt(d.qkv_dtype)),
+        *toks, int(j), _ptr(o, "o", NH * d.dv, torch.float32), ctypes.c_void_p(_stream(stream))))
+
+
+def sketchssm_fullread_decode(d: sketchssm_dims, S, q, k, v, alpha, beta, o, stream=None):
+    """Baseline decode step: read, update and write the full state; o = S^T q."""
+    NH = d.B * d.H
+    toks = _token_ptrs(d, 1, k, v, alpha, beta)
+    _check("sketchssm_fullread_decode", library().sketchssm_fullread_decode(
+        ctypes.byref(d), _ptr(S, "S", NH * d.dv * d.dk, _dt(d.state_dtype)),
+        _ptr(q, "q", NH * d.dk, _dt(d.qkv_dtype)), *toks, _ptr(o, "o", NH * d.dv, torch.float32),
+        ctypes.c_void_p(_stream(stream))))
+
+
+def sketchssm_calibrate_workspace_bytes(d: sketchssm_dims, Nq: int, Ns: int) -> int:
+    return int(library().sketchssm_calibrate_workspace_bytes(ctypes.byref(d), int(Nq), int(Ns)))
+
+
+def sketchssm_calibrate_basis(d: sketchssm_dims, q_cal, S_cal, U, R, workspace=None, ridge: float = 1e-8,
+                              stream=None):
+    """Offline basis: q_cal [H,Nq,dk] fp32, S_cal [Ns,H,dv,dk] -> U [H,dk,r], R [H,r,dk].
+
+    `workspace` is a uint8 CUDA tensor of at least sketchssm_calibrate_workspace_bytes bytes; when
+    None, one is allocated here through torch (the library itself never allocates).
+    """
+    Nq = q_cal.shape[1]
+    Ns = S_cal.shape[0]
+    need = sketchssm_calibrate_workspace_bytes(d, Nq, Ns)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q_cal.device)
+    _check("sketchssm_calibrate_basis", library().sketchssm_calibrate_basis(
+        ctypes.byref(d), _ptr(q_cal, "q_cal", d.H * Nq * d.dk, torch.float32), int(Nq),
+        _ptr(S_cal, "S_cal", Ns * d.H * d.dv * d.dk, _dt(d.state_dtype)), int(Ns), float(ridge),
+        _ptr(U, "U", d.H * d.dk * d.r, torch.float32), _ptr(R, "R", d.H * d.r * d.dk, torch.float32),
+        _ptr(workspace, "workspace"), ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+        ctypes.c_void_p(_stream(stream))))

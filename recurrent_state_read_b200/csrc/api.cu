@@ -1,0 +1,116 @@
+// api.cu -- the exported C ABI (include/sketchssm.h): host-side validation, then launch.
+//
+// Every entry point checks its arguments before touching the GPU and returns a
+// sketchssm_status; nothing is launched on error.  No entry point allocates.
+#include <stdint.h>
+
+#include "internal.h"
+
+using namespace skssm;
+
+namespace {
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int check_dims(const sketchssm_dims *d) {
+    if (!d) return SKSSM_ERR_NULL;
+    if (d->kind < SKSSM_MAMBA2 || d->kind > SKSSM_KDA) return SKSSM_ERR_DIMS;
+    if (d->state_dtype != SKSSM_F32 && d->state_dtype != SKSSM_BF16) return SKSSM_ERR_DTYPE;
+    if (d->qkv_dtype != SKSSM_F32 && d->qkv_dtype != SKSSM_BF16) return SKSSM_ERR_DTYPE;
+    if (d->dk != 64 && d->dk != 128) return SKSSM_ERR_DIMS;
+    if (d->dv != 64 && d->dv != 128) return SKSSM_ERR_DIMS;
+    if (!((d->r >= 1 && d->r <= 32) || d->r == d->dk)) return SKSSM_ERR_DIMS;
+    if (d->W < 1 || d->W > 64) return SKSSM_ERR_DIMS;
+    if (d->B < 1 || d->H < 1) return SKSSM_ERR_DIMS;
+    if ((int64_t)d->B * d->H >= (int64_t)1 << 31) return SKSSM_ERR_DIMS;
+    return SKSSM_OK;
+}
+
+// window buffer / token pointers: k, v 16 B; alpha, beta 4 B
+int check_tokens(const sketchssm_dims *d, const void *k, const void *v, const float *alpha,
+                 const float *beta) {
+    if (!k || !v || !alpha) return SKSSM_ERR_NULL;
+    if (d->kind != SKSSM_MAMBA2 && !beta) return SKSSM_ERR_NULL;
+    if (!aligned(k, 16) || !aligned(v, 16) || !aligned(alpha, 4)) return SKSSM_ERR_ALIGN;
+    if (beta && !aligned(beta, 4)) return SKSSM_ERR_ALIGN;
+    if (d->kind == SKSSM_KDA && !aligned(alpha, 16)) return SKSSM_ERR_ALIGN;
+    return SKSSM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *sketchssm_status_string(int status) {
+    switch (status) {
+        case SKSSM_OK: return "ok";
+        case SKSSM_ERR_NULL: return "a required pointer is NULL";
+        case SKSSM_ERR_DIMS: return "unsupported kind or sizes";
+        case SKSSM_ERR_RANGE: return "step, token count or calibration count out of range";
+        case SKSSM_ERR_ALIGN: return "a pointer breaks its alignment rule";
+        case SKSSM_ERR_DTYPE: return "unsupported storage dtype";
+        case SKSSM_ERR_CUDA: return "CUDA launch or runtime call failed";
+        case SKSSM_ERR_WORKSPACE: return "workspace missing or too small";
+        default: return "unknown status";
+    }
+}
+
+int sketchssm_version(void) { return 10000; }
+
+int sketchssm_update_window(const sketchssm_dims *d, void *S, float *P, const float *U, const void *k,
+                            const void *v, const float *alpha, const float *beta, int n_tokens,
+                            void *stream) {
+    int rc = check_dims(d);
+    if (rc) return rc;
+    if (!S || !P || !U) return SKSSM_ERR_NULL;
+    if (n_tokens < 0 || n_tokens > d->W) return SKSSM_ERR_RANGE;
+    if (n_tokens > 0 && (rc = check_tokens(d, k, v, alpha, beta))) return rc;
+    if (!aligned(S, 16) || !aligned(P, 16) || !aligned(U, 16)) return SKSSM_ERR_ALIGN;
+    return launch_update_window(*d, S, P, U, k, v, alpha, beta, n_tokens, (cudaStream_t)stream);
+}
+
+int sketchssm_decode_step(const sketchssm_dims *d, const float *P, const float *R, const void *q,
+                          const void *k, const void *v, const float *alpha, const float *beta, int j,
+                          float *o, void *stream) {
+    int rc = check_dims(d);
+    if (rc) return rc;
+    if (!P || !R || !q || !o) return SKSSM_ERR_NULL;
+    if (j < 1 || j > d->W) return SKSSM_ERR_RANGE;
+    if ((rc = check_tokens(d, k, v, alpha, beta))) return rc;
+    if (!aligned(P, 16) || !aligned(R, 16) || !aligned(q, 16) || !aligned(o, 16)) return SKSSM_ERR_ALIGN;
+    return launch_decode_step(*d, P, R, q, k, v, alpha, beta, j, o, (cudaStream_t)stream);
+}
+
+int sketchssm_fullread_decode(const sketchssm_dims *d, void *S, const void *q, const void *k,
+                              const void *v, const float *alpha, const float *beta, float *o,
+                              void *stream) {
+    int rc = check_dims(d);
+    if (rc) return rc;
+    if (!S || !q || !o) return SKSSM_ERR_NULL;
+    if ((rc = check_tokens(d, k, v, alpha, beta))) return rc;
+    if (!aligned(S, 16) || !aligned(q, 16) || !aligned(o, 16)) return SKSSM_ERR_ALIGN;
+    return launch_fullread(*d, S, q, k, v, alpha, beta, o, (cudaStream_t)stream);
+}
+
+size_t sketchssm_calibrate_workspace_bytes(const sketchssm_dims *d, int Nq, int Ns) {
+    if (check_dims(d) != SKSSM_OK || Nq < 1 || Ns < 1) return 0;
+    return calibrate_workspace_bytes(*d, Nq, Ns);
+}
+
+int sketchssm_calibrate_basis(const sketchssm_dims *d, const float *q_cal, int Nq, const void *S_cal,
+                              int Ns, double ridge, float *U, float *R, void *workspace,
+                              size_t workspace_bytes, void *stream) {
+    int rc = check_dims(d);
+    if (rc) return rc;
+    if (!q_cal || !S_cal || !U || !R) return SKSSM_ERR_NULL;
+    if (Nq < 1 || Ns < 1 || !(ridge >= 0.0)) return SKSSM_ERR_RANGE;
+    if ((int64_t)Ns * d->dv >= (int64_t)1 << 31 || (int64_t)Nq * d->H >= (int64_t)1 << 31)
+        return SKSSM_ERR_RANGE;
+    if (!workspace || workspace_bytes < calibrate_workspace_bytes(*d, Nq, Ns)) return SKSSM_ERR_WORKSPACE;
+    if (!aligned(q_cal, 16) || !aligned(S_cal, 16) || !aligned(U, 16) || !aligned(R, 16) ||
+        !aligned(workspace, 256))
+        return SKSSM_ERR_ALIGN;
+    return launch_calibrate(*d, q_cal, Nq, S_cal, Ns, ridge, U, R, workspace, (cudaStream_t)stream);
+}
+
+}  // extern "C"

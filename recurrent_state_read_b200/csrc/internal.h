@@ -1,0 +1,58 @@
+// internal.h -- launchers behind the C ABI (not exported).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <type_traits>
+
+#include "sketchssm.h"
+
+namespace skssm {
+
+// Call fn(kind, dk, state type, qkv type) with compile-time constants for the
+// supported combinations; returns SKSSM_ERR_DIMS / SKSSM_ERR_DTYPE otherwise.
+template <typename Fn>
+int dispatch(const sketchssm_dims &d, Fn &&fn) {
+    auto by_q = [&](auto K, auto D, auto S) -> int {
+        if (d.qkv_dtype == SKSSM_F32) return fn(K, D, S, (float *)nullptr);
+        if (d.qkv_dtype == SKSSM_BF16) return fn(K, D, S, (__nv_bfloat16 *)nullptr);
+        return SKSSM_ERR_DTYPE;
+    };
+    auto by_s = [&](auto K, auto D) -> int {
+        if (d.state_dtype == SKSSM_F32) return by_q(K, D, (float *)nullptr);
+        if (d.state_dtype == SKSSM_BF16) return by_q(K, D, (__nv_bfloat16 *)nullptr);
+        return SKSSM_ERR_DTYPE;
+    };
+    auto by_d = [&](auto K) -> int {
+        if (d.dk == 64) return by_s(K, std::integral_constant<int, 64>());
+        if (d.dk == 128) return by_s(K, std::integral_constant<int, 128>());
+        return SKSSM_ERR_DIMS;
+    };
+    switch (d.kind) {
+        case SKSSM_MAMBA2: return by_d(std::integral_constant<int, 0>());
+        case SKSSM_GDN: return by_d(std::integral_constant<int, 1>());
+        case SKSSM_KDA: return by_d(std::integral_constant<int, 2>());
+        default: return SKSSM_ERR_DIMS;
+    }
+}
+
+inline int launch_status() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SKSSM_OK : SKSSM_ERR_CUDA;
+}
+
+int launch_update_window(const sketchssm_dims &d, void *S, float *P, const float *U, const void *k,
+                         const void *v, const float *alpha, const float *beta, int n_tokens,
+                         cudaStream_t stream);
+int launch_fullread(const sketchssm_dims &d, void *S, const void *q, const void *k, const void *v,
+                    const float *alpha, const float *beta, float *o, cudaStream_t stream);
+int launch_decode_step(const sketchssm_dims &d, const float *P, const float *R, const void *q,
+                       const void *k, const void *v, const float *alpha, const float *beta, int j,
+                       float *o, cudaStream_t stream);
+
+size_t calibrate_workspace_bytes(const sketchssm_dims &d, int Nq, int Ns);
+int launch_calibrate(const sketchssm_dims &d, const float *q_cal, int Nq, const void *S_cal, int Ns,
+                     double ridge, float *U, float *R, void *workspace, cudaStream_t stream);
+
+}  // namespace skssm

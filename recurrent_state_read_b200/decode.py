@@ -1,0 +1,85 @@
+"""The SketchSSM decode schedule on the GPU, composed from the C entry points.
+
+Timeline (SketchSSM abstract and the agihunt digest's "Mechanism details"):
+within a window of W steps the state is fixed; step j reads the sketch and the
+buffered tokens 1..j; after the window's last step one kernel applies the W
+buffered tokens to the state and refreshes the sketch.  The full-read baseline
+updates and reads the whole state at every step.  This module is host-side
+control flow only: every arithmetic step runs in libsketchssm.so.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import torch
+
+from . import (sketchssm_decode_step, sketchssm_dims, sketchssm_fullread_decode,
+               sketchssm_update_window)
+
+
+@dataclasses.dataclass
+class WindowBuffer:
+    """Device window buffer, time-major: k [W,B,H,dk], v [W,B,H,dv], alpha [W,B,H(,dk)],
+    beta [W,B,H] (None for Mamba-2), q [W,B,H,dk] (the queries of the window's steps)."""
+    k: torch.Tensor
+    v: torch.Tensor
+    alpha: torch.Tensor
+    beta: Optional[torch.Tensor]
+    q: Optional[torch.Tensor] = None
+
+    @staticmethod
+    def empty(d: sketchssm_dims, device="cuda", with_query=True) -> "WindowBuffer":
+        qt = torch.float32 if d.qkv_dtype == 0 else torch.bfloat16
+        W, B, H = d.W, d.B, d.H
+        a_shape = (W, B, H, d.dk) if d.kind == 2 else (W, B, H)
+        return WindowBuffer(
+            k=torch.empty(W, B, H, d.dk, dtype=qt, device=device),
+            v=torch.empty(W, B, H, d.dv, dtype=qt, device=device),
+            alpha=torch.empty(a_shape, dtype=torch.float32, device=device),
+            beta=None if d.kind == 0 else torch.empty(W, B, H, dtype=torch.float32, device=device),
+            q=torch.empty(W, B, H, d.dk, dtype=qt, device=device) if with_query else None,
+        )
+
+    def fill(self, tok: dict, n: Optional[int] = None):
+        """Copy tokens (dict of [n,B,H,...] tensors) into slots 0..n-1."""
+        n = tok["k"].shape[0] if n is None else n
+        for name in ("k", "v", "alpha", "beta", "q"):
+            dst = getattr(self, name)
+            if dst is not None and tok.get(name) is not None:
+                dst[:n].copy_(tok[name][:n], non_blocking=True)
+
+
+def sketch_window(d: sketchssm_dims, S, P, U, R, buf: WindowBuffer, out, n: Optional[int] = None,
+                  stream=None):
+    """One window of the sketch path: n decode steps (outputs into out[0..n-1], each [B,H,dv]
+    fp32) read the sketch; then one window update applies the n tokens and refreshes P."""
+    n = d.W if n is None else n
+    for j in range(1, n + 1):
+        sketchssm_decode_step(d, P, R, buf.q[j - 1], buf.k, buf.v, buf.alpha, buf.beta, j, out[j - 1],
+                              stream)
+    sketchssm_update_window(d, S, P, U, buf.k, buf.v, buf.alpha, buf.beta, n, stream)
+
+
+def fullread_window(d: sketchssm_dims, S, buf: WindowBuffer, out, n: Optional[int] = None, stream=None):
+    """n steps of the full-read baseline over the same window buffer."""
+    n = d.W if n is None else n
+    for t in range(n):
+        sketchssm_fullread_decode(d, S, buf.q[t], buf.k[t], buf.v[t], buf.alpha[t],
+                                  None if buf.beta is None else buf.beta[t], out[t], stream)
+
+
+def prefill(d: sketchssm_dims, S, P, U, token_source, n_tokens: int, stream=None):
+    """Advance S through n_tokens tokens with window updates of up to W tokens each.
+
+    token_source(t0, n) returns a dict of device tensors [n,B,H,...] for tokens t0..t0+n-1.
+    P is refreshed as a by-product (the last refresh is the sketch of the final state).
+    """
+    buf = WindowBuffer.empty(d, device=S.device, with_query=False)
+    for t0 in range(0, n_tokens, d.W):
+        n = min(d.W, n_tokens - t0)
+        buf.fill(token_source(t0, n), n)
+        sketchssm_update_window(d, S, P, U, buf.k, buf.v, buf.alpha, buf.beta, n, stream)
+    if n_tokens == 0:
+        sketchssm_update_window(d, S, P, U, None, None, None, None, 0, stream)

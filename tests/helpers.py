@@ -1,0 +1,71 @@
+"""Shared test helpers: layout conversion, error metrics, tolerances, input builders.
+
+Tolerances.  The workload contract fixes: updated fp32 state within a max
+relative error of 1e-5; sketch-path outputs within a relative L2 error of 2e-3.
+Relative error of a state is measured per head as max|S_gpu - S_ref| / max|S_ref|
+(elementwise relative error is meaningless near zero) and the worst head is
+reported.  Both sides read identical bf16-rounded inputs; the GPU accumulates in
+fp32, so the observed errors are ~1e-6.  The tests also hold the GPU to a
+tighter fp32-derived bound (TIGHT_*): dot products of <= 128 terms and <= 64
+sequential updates, each adding O(1e-7) relative error, stay below 1e-4.
+bf16 storage (the sweep) has no contracted tolerance; bf16 spacing is 2^-8 of
+the value, so states are held to 1e-2 and outputs to 1e-2 (soft gate).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+STATE_TOL = 1e-5   # contract: fp32 state, max relative error
+OUT_TOL = 2e-3     # contract: sketch-path outputs, relative L2
+TIGHT_OUT = 1e-4   # fp32-derived bound on outputs (both paths)
+BF16_STATE_TOL = 1e-2
+BF16_OUT_TOL = 1e-2
+
+
+def to_logical(S_gpu: torch.Tensor, heads=None) -> np.ndarray:
+    """GPU state [B,H,dv,dk] (any dtype) -> oracle layout [N,dk,dv] float64 (optionally sampled heads)."""
+    B, H, dv, dk = S_gpu.shape
+    S = S_gpu.reshape(B * H, dv, dk)
+    if heads is not None:
+        S = S[torch.as_tensor(heads, device=S.device)]
+    return S.transpose(1, 2).double().cpu().numpy()
+
+
+def to_gpu_state(S_log: np.ndarray, B: int, H: int, dtype=torch.float32, device="cuda") -> torch.Tensor:
+    """Oracle layout [N,dk,dv] -> GPU state [B,H,dv,dk] (rounded to dtype)."""
+    N, dk, dv = S_log.shape
+    t = torch.from_numpy(np.ascontiguousarray(S_log.transpose(0, 2, 1)))
+    return t.to(dtype).reshape(B, H, dv, dk).contiguous().to(device)
+
+
+def flat_tokens(tok: dict, heads=None) -> dict:
+    """[T,B,H,...] token tensors -> [T,N,...] float64 numpy (optionally sampled flat heads)."""
+    out = {}
+    for key, val in tok.items():
+        if val is None:
+            out[key] = None
+            continue
+        T, B, H = val.shape[:3]
+        x = val.reshape(T, B * H, *val.shape[3:])
+        if heads is not None:
+            x = x[:, torch.as_tensor(heads, device=x.device)]
+        out[key] = x.double().cpu().numpy()
+    return out
+
+
+def state_err(S_gpu_log: np.ndarray, S_ref: np.ndarray) -> float:
+    num = np.abs(S_gpu_log - S_ref).reshape(S_ref.shape[0], -1).max(1)
+    den = np.abs(S_ref).reshape(S_ref.shape[0], -1).max(1)
+    return float((num / np.maximum(den, 1e-300)).max())
+
+
+def rel_l2(a, b) -> float:
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def to_device(tok: dict, device="cuda") -> dict:
+    return {k: (None if v is None else v.to(device).contiguous()) for k, v in tok.items()}

@@ -1,0 +1,79 @@
+"""GPU offline calibration (sketchssm_calibrate_basis) against the oracle's.
+
+The two sides take different routes (the GPU: Cholesky of G, Jacobi on
+L^T C L, U = L^-T V_r; the oracle: symmetric square roots from numpy's eigh and
+a generic solve), so their U need not agree column by column; what any valid
+answer must share is the G-weighted projector U R, the identity R U = I and the
+calibration objective.  The calibration states are the oracle's prefill states
+of seeded calibration sequences; the queries come from the workload generator.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+from oracle import calibration as cal
+from tests.helpers import flat_tokens, to_gpu_state
+
+pytestmark = pytest.mark.gpu
+
+
+def _cal_inputs(cfg, n_seq, n_tokens, n_q):
+    tok = flat_tokens(wl.token_block(cfg, "cal", 0, n_tokens, B=n_seq))
+    S = np.zeros((n_seq * cfg.H, cfg.dk, cfg.dv))
+    S, _ = oracle.exact_steps(cfg.kind, S, tok["k"], tok["v"], tok["alpha"], tok["beta"])
+    S = S.astype(np.float32).astype(np.float64)
+    q = wl.calibration_queries(cfg, n=n_q)
+    return S.reshape(n_seq, cfg.H, cfg.dk, cfg.dv), q
+
+
+@pytest.mark.parametrize("cid,n_seq,n_tokens,n_q,r", [
+    (0, 64, 128, 1024, 8),     # the tiny Mamba-2 case with its full calibration recipe
+    (2, 16, 64, 1024, 8),      # GDN shape, reduced calibration set
+    (3, 16, 64, 1024, 16),     # KDA shape
+    (1, 8, 64, 1024, 4),       # Mamba-2 dk=128, dv=64
+    (2, 8, 32, 512, 128),      # complete basis: U R = I
+])
+def test_calibrate_matches_oracle(cid, n_seq, n_tokens, n_q, r):
+    import recurrent_state_read_b200 as rs
+
+    cfg = wl.workload(cid, H=min(wl.CONFIGS[cid].H, 6), r=r)
+    S_cal, q_cal = _cal_inputs(cfg, n_seq, n_tokens, n_q)
+    U_ref, R_ref = oracle.calibrate_heads(S_cal, q_cal.double().numpy(), r)
+    d = rs.dims(cfg.kind, n_seq, cfg.H, cfg.dk, cfg.dv, r, cfg.W, torch.float32, cfg.torch_qkv_dtype)
+    S_gpu = to_gpu_state(S_cal.reshape(n_seq * cfg.H, cfg.dk, cfg.dv), n_seq, cfg.H)
+    U = torch.full((cfg.H, cfg.dk, r), float("nan"), device="cuda")
+    R = torch.full((cfg.H, r, cfg.dk), float("nan"), device="cuda")
+    rs.sketchssm_calibrate_basis(d, q_cal.cuda().contiguous(), S_gpu, U, R)
+    torch.cuda.synchronize()
+    U, R = U.double().cpu().numpy(), R.double().cpu().numpy()
+    for h in range(cfg.H):
+        Pi, Pi_ref = U[h] @ R[h], U_ref[h] @ R_ref[h]
+        scale = max(1.0, np.abs(Pi_ref).max())
+        assert np.abs(Pi - Pi_ref).max() <= 1e-5 * scale, (h, np.abs(Pi - Pi_ref).max())
+        np.testing.assert_allclose(R[h] @ U[h], np.eye(r), atol=1e-5)
+        G = cal.gram_states(S_cal[:, h])
+        C = cal.gram_queries(q_cal[h].double().numpy())
+        j_gpu, j_ref = cal.objective(G, C, U[h], R[h]), cal.objective(G, C, U_ref[h], R_ref[h])
+        assert j_gpu <= j_ref * (1 + 1e-4) + 1e-12 * np.trace(G @ C), (h, j_gpu, j_ref)
+
+
+def test_calibrate_bf16_states():
+    import recurrent_state_read_b200 as rs
+
+    cfg = wl.workload(2, H=3, r=8)
+    S_cal, q_cal = _cal_inputs(cfg, 16, 64, 512)
+    S_cal = oracle.round_bf16(S_cal)
+    U_ref, R_ref = oracle.calibrate_heads(S_cal, q_cal.double().numpy(), 8)
+    d = rs.dims("gdn", 16, cfg.H, 128, 128, 8, 16, torch.bfloat16, torch.bfloat16)
+    S_gpu = to_gpu_state(S_cal.reshape(-1, 128, 128), 16, cfg.H, torch.bfloat16)
+    U = torch.empty(cfg.H, 128, 8, device="cuda")
+    R = torch.empty(cfg.H, 8, 128, device="cuda")
+    rs.sketchssm_calibrate_basis(d, q_cal.cuda().contiguous(), S_gpu, U, R)
+    torch.cuda.synchronize()
+    for h in range(cfg.H):
+        Pi = U[h].double().cpu().numpy() @ R[h].double().cpu().numpy()
+        Pi_ref = U_ref[h] @ R_ref[h]
+        assert np.abs(Pi - Pi_ref).max() <= 1e-5 * max(1.0, np.abs(Pi_ref).max())

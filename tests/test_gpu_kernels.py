@@ -1,0 +1,194 @@
+"""GPU parity of each kernel alone, through the C ABI, against the fp64 oracle.
+
+Inputs: seeded tokens from the workload generator at reduced batch (B=3, H=5,
+a ragged 15 heads), seeded Gaussian states, bases and coefficient maps; both
+sides see the same values.  Each case isolates one kernel: the window update
+is fed the same window-start state as the oracle, the decode step the same
+sketch.  Sizes and edge cases: every kind, dk/dv in {64,128}, fp32/bf16 state
+and q/k/v, r from 1 to 32 and r = dk, n_tokens = 0 (sketch refresh only),
+partial and full windows, W = 1 and W = 64.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+from tests.helpers import (BF16_OUT_TOL, BF16_STATE_TOL, STATE_TOL, TIGHT_OUT, flat_tokens, rel_l2,
+                           state_err, to_device, to_gpu_state, to_logical)
+
+pytestmark = pytest.mark.gpu
+
+KIND_CFG = {"mamba2": 1, "gdn": 2, "kda": 3}
+
+
+def _setup(kind, dk, dv, r, W, sdt, qdt, B=3, H=5, seed=0):
+    import recurrent_state_read_b200 as rs
+
+    cfg = wl.workload(KIND_CFG[kind], B=B, H=H, dk=dk, dv=dv, r=r, W=W,
+                      qkv_dtype="f32" if qdt == torch.float32 else "bf16",
+                      state_dtype="f32" if sdt == torch.float32 else "bf16",
+                      q_rank=min(8, dk))
+    d = rs.dims(kind, B, H, dk, dv, r, W, sdt, qdt)
+    g = torch.Generator().manual_seed(1000 + seed)
+    S0 = torch.randn(B * H, dk, dv, generator=g, dtype=torch.float64).numpy()
+    S0 = oracle.round_bf16(S0) if sdt == torch.bfloat16 else S0.astype(np.float32).astype(np.float64)
+    U = torch.randn(H, dk, r, generator=g) / dk ** 0.5
+    R = torch.randn(H, r, dk, generator=g) / dk ** 0.5
+    tok = wl.token_block(cfg, "decode", 0, W, with_query=True)
+    return cfg, d, S0, U, R, tok
+
+
+CASES = [
+    # kind, dk, dv, r, W, state dtype, qkv dtype
+    ("mamba2", 128, 64, 8, 16, torch.float32, torch.bfloat16),
+    ("gdn", 128, 128, 8, 16, torch.float32, torch.bfloat16),
+    ("kda", 128, 128, 8, 16, torch.float32, torch.bfloat16),
+    ("mamba2", 64, 64, 8, 8, torch.float32, torch.float32),
+    ("gdn", 64, 128, 4, 5, torch.float32, torch.float32),
+    ("kda", 128, 64, 16, 7, torch.float32, torch.bfloat16),
+    ("gdn", 128, 128, 32, 32, torch.float32, torch.bfloat16),
+    ("gdn", 128, 128, 13, 4, torch.float32, torch.bfloat16),
+    ("mamba2", 128, 64, 1, 1, torch.float32, torch.bfloat16),
+    ("kda", 64, 64, 64, 3, torch.float32, torch.float32),      # r == dk
+    ("gdn", 128, 128, 8, 64, torch.float32, torch.bfloat16),   # longest window
+    ("mamba2", 128, 64, 8, 16, torch.bfloat16, torch.bfloat16),
+    ("gdn", 128, 128, 8, 16, torch.bfloat16, torch.bfloat16),
+    ("kda", 128, 128, 8, 16, torch.bfloat16, torch.bfloat16),
+    ("gdn", 64, 64, 4, 8, torch.bfloat16, torch.float32),
+]
+
+
+def _ids(c):
+    return f"{c[0]}-dk{c[1]}-dv{c[2]}-r{c[3]}-W{c[4]}-S{str(c[5])[6:]}-q{str(c[6])[6:]}"
+
+
+@pytest.mark.parametrize("case", CASES, ids=[_ids(c) for c in CASES])
+def test_update_window(case):
+    import recurrent_state_read_b200 as rs
+
+    kind, dk, dv, r, W, sdt, qdt = case
+    cfg, d, S0, U, R, tok = _setup(kind, dk, dv, r, W, sdt, qdt)
+    B, H = d.B, d.H
+    heads = np.arange(B * H)
+    Uh = oracle.per_head(U, H, heads)
+    ft = flat_tokens(tok)
+    dev = to_device(tok)
+    for n in sorted({0, 1, max(1, W // 2), W}):
+        S = to_gpu_state(S0, B, H, sdt)
+        P = torch.full((B, H, dv, r), float("nan"), device="cuda")
+        rs.sketchssm_update_window(d, S, P, U.cuda(), dev["k"], dev["v"], dev["alpha"], dev["beta"], n)
+        torch.cuda.synchronize()
+        sl = slice(0, n)
+        Sref, Pref = oracle.update_window(kind, S0, Uh, ft["k"][sl] if n else None, ft["v"][sl],
+                                          ft["alpha"][sl], None if ft["beta"] is None else ft["beta"][sl],
+                                          bf16_state=sdt == torch.bfloat16)
+        tol = STATE_TOL if sdt == torch.float32 else BF16_STATE_TOL
+        es = state_err(to_logical(S), Sref)
+        ep = state_err(P.reshape(B * H, dv, r).double().cpu().numpy(), Pref)
+        assert es <= tol, (n, es)
+        assert ep <= tol, (n, ep)
+        if n == 0:  # a sketch refresh leaves the state untouched, bit for bit
+            assert torch.equal(S, to_gpu_state(S0, B, H, sdt))
+
+
+@pytest.mark.parametrize("case", CASES, ids=[_ids(c) for c in CASES])
+def test_decode_step(case):
+    import recurrent_state_read_b200 as rs
+
+    kind, dk, dv, r, W, sdt, qdt = case
+    cfg, d, S0, U, R, tok = _setup(kind, dk, dv, r, W, sdt, qdt, seed=1)
+    B, H = d.B, d.H
+    heads = np.arange(B * H)
+    g = torch.Generator().manual_seed(7)
+    P = torch.randn(B, H, dv, r, generator=g)
+    ft = flat_tokens(tok)
+    dev = to_device(tok)
+    Rh = oracle.per_head(R, H, heads)
+    for j in sorted({1, max(1, W // 2), W}):
+        o = torch.full((B, H, dv), float("nan"), device="cuda")
+        rs.sketchssm_decode_step(d, P.cuda(), R.cuda(), dev["q"][j - 1], dev["k"], dev["v"], dev["alpha"],
+                                 dev["beta"], j, o)
+        torch.cuda.synchronize()
+        sl = slice(0, j)
+        ref = oracle.sketch_read(kind, P.reshape(B * H, dv, r), Rh, ft["q"][j - 1], ft["k"][sl], ft["v"][sl],
+                                 ft["alpha"][sl], None if ft["beta"] is None else ft["beta"][sl])
+        err = rel_l2(o.reshape(B * H, dv).cpu(), ref)
+        assert err <= TIGHT_OUT, (j, err)
+
+
+@pytest.mark.parametrize("case", CASES, ids=[_ids(c) for c in CASES])
+def test_fullread_decode(case):
+    import recurrent_state_read_b200 as rs
+
+    kind, dk, dv, r, W, sdt, qdt = case
+    cfg, d, S0, U, R, tok = _setup(kind, dk, dv, r, W, sdt, qdt, seed=2)
+    B, H = d.B, d.H
+    ft = flat_tokens(tok)
+    dev = to_device(tok)
+    S = to_gpu_state(S0, B, H, sdt)
+    T = min(W, 6)
+    outs = torch.full((T, B, H, dv), float("nan"), device="cuda")
+    for t in range(T):
+        rs.sketchssm_fullread_decode(d, S, dev["q"][t], dev["k"][t], dev["v"][t], dev["alpha"][t],
+                                     None if dev["beta"] is None else dev["beta"][t], outs[t])
+    torch.cuda.synchronize()
+    sl = slice(0, T)
+    Sref, Oref = oracle.exact_steps(kind, S0, ft["k"][sl], ft["v"][sl], ft["alpha"][sl],
+                                    None if ft["beta"] is None else ft["beta"][sl], ft["q"][sl],
+                                    bf16_state=sdt == torch.bfloat16)
+    bf = sdt == torch.bfloat16
+    assert state_err(to_logical(S), Sref) <= (BF16_STATE_TOL if bf else STATE_TOL)
+    assert rel_l2(outs.reshape(T, B * H, dv).cpu(), Oref) <= (BF16_OUT_TOL if bf else TIGHT_OUT)
+
+
+def test_complete_basis_sketch_is_exact_read():
+    """r = dk with U = R = I: decode-step outputs equal the full-read outputs (GPU both sides)."""
+    import recurrent_state_read_b200 as rs
+
+    kind, dk, dv, W = "gdn", 64, 64, 8
+    cfg, d, S0, U, R, tok = _setup(kind, dk, dv, dk, W, torch.float32, torch.float32)
+    B, H = d.B, d.H
+    eye = torch.eye(dk).expand(H, dk, dk).contiguous().cuda()
+    dev = to_device(tok)
+    S = to_gpu_state(S0, B, H)
+    Sf = S.clone()
+    P = torch.empty(B, H, dv, dk, device="cuda")
+    rs.sketchssm_update_window(d, S, P, eye, None, None, None, None, 0)
+    o_s = torch.empty(W, B, H, dv, device="cuda")
+    o_f = torch.empty(W, B, H, dv, device="cuda")
+    for j in range(1, W + 1):
+        rs.sketchssm_decode_step(d, P, eye, dev["q"][j - 1], dev["k"], dev["v"], dev["alpha"], dev["beta"],
+                                 j, o_s[j - 1])
+        rs.sketchssm_fullread_decode(d, Sf, dev["q"][j - 1], dev["k"][j - 1], dev["v"][j - 1],
+                                     dev["alpha"][j - 1], dev["beta"][j - 1], o_f[j - 1])
+    torch.cuda.synchronize()
+    assert rel_l2(o_s.cpu(), o_f.cpu()) <= TIGHT_OUT
+
+
+def test_invalid_arguments_launch_nothing():
+    import recurrent_state_read_b200 as rs
+
+    d = rs.dims("gdn", 2, 2, 128, 128, 8, 16)
+    S = torch.zeros(2, 2, 128, 128, device="cuda")
+    P = torch.zeros(2, 2, 128, 8, device="cuda")
+    U = torch.zeros(2, 128, 8, device="cuda")
+    k = torch.zeros(17, 2, 2, 128, dtype=torch.bfloat16, device="cuda")  # room for 17 slots
+    a = torch.zeros(17, 2, 2, device="cuda")
+    with pytest.raises(rs.SketchSSMError) as e:
+        rs.sketchssm_update_window(d, S, P, U, k, k, a, a, 17)  # W = 16
+    assert e.value.status == -3
+    with pytest.raises(rs.SketchSSMError) as e:
+        rs.sketchssm_update_window(d, S, P, U, k, k, a, None, 4)  # GDN needs beta
+    assert e.value.status == -1
+    bad = rs.dims("gdn", 2, 2, 96, 128, 8, 16)
+    with pytest.raises(rs.SketchSSMError) as e:
+        rs.sketchssm_update_window(bad, S, P, U, k, k, a, a, 4)
+    assert e.value.status == -2
+    o = torch.zeros(2, 2, 128, device="cuda")
+    with pytest.raises(rs.SketchSSMError) as e:
+        rs.sketchssm_decode_step(d, P, U, k[0], k, k, a, a, 0, o)
+    assert e.value.status == -3
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(S) == 0 and torch.count_nonzero(P) == 0

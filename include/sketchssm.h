@@ -179,6 +179,31 @@ int sketchssm_calibrate_basis(const sketchssm_dims *dims, const float *q_cal, in
                               const void *S_cal, int Ns, double ridge, float *U, float *R,
                               void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * sketchssm_calibrate_basis_noalloc -- sketchssm_calibrate_basis without a
+ * workspace argument, for callers that cannot allocate device memory when they
+ * calibrate (an engine that gave all free memory to its own pool at start-up,
+ * a plug-in under a memory budget set by its host application, code that
+ * cannot accept the device synchronisation of cudaFree).  The SketchSSM pages
+ * have no counterpart: this is a deployment convenience, not part of the method.
+ * Same inputs, outputs and results as sketchssm_calibrate_basis.
+ *   Scratch: a fixed 3 MiB array inside the library's device image, held on
+ *   every GPU that loads the library until the process exits.  One pass covers
+ *   up to 8 heads at dk = 128 (32 at dk = 64); more heads run as several passes,
+ *   in order on `stream`.  A size whose single head does not fit the scratch is
+ *   rejected with SKSSM_ERR_WORKSPACE (no supported dk reaches that limit).
+ *   Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ *   The first call on a device looks up the scratch's device address (once per
+ *   device, with that device current); make that first call before any stream
+ *   capture.  All calls share the one scratch array, which keeps the last call's
+ *   contents (every pass overwrites what it reads, so nothing needs clearing);
+ *   calls that overlap on the GPU race on it and must be ordered by the caller.
+ * Errors: as sketchssm_calibrate_basis (ERR_WORKSPACE as above).
+ */
+int sketchssm_calibrate_basis_noalloc(const sketchssm_dims *dims, const float *q_cal, int Nq,
+                                      const void *S_cal, int Ns, double ridge, float *U, float *R,
+                                      void *stream);
+
 #ifdef __cplusplus
 }
 #endif

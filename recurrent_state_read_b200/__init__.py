@@ -34,6 +34,7 @@ EXPORTS = (
     "sketchssm_fullread_decode",
     "sketchssm_calibrate_workspace_bytes",
     "sketchssm_calibrate_basis",
+    "sketchssm_calibrate_basis_noalloc",
 )
 
 
@@ -76,8 +77,9 @@ def library() -> ctypes.CDLL:
         lib.sketchssm_calibrate_workspace_bytes.restype = ctypes.c_size_t
         lib.sketchssm_calibrate_basis.argtypes = [D, P, i, P, i, ctypes.c_double, P, P, P,
                                                   ctypes.c_size_t, P]
+        lib.sketchssm_calibrate_basis_noalloc.argtypes = [D, P, i, P, i, ctypes.c_double, P, P, P]
         for f in ("sketchssm_update_window", "sketchssm_decode_step", "sketchssm_fullread_decode",
-                  "sketchssm_calibrate_basis"):
+                  "sketchssm_calibrate_basis", "sketchssm_calibrate_basis_noalloc"):
             getattr(lib, f).restype = i
         _lib = lib
     return _lib
@@ -180,4 +182,17 @@ def sketchssm_calibrate_basis(d: sketchssm_dims, q_cal, S_cal, U, R, workspace=N
         _ptr(S_cal, "S_cal", Ns * d.H * d.dv * d.dk, _dt(d.state_dtype)), int(Ns), float(ridge),
         _ptr(U, "U", d.H * d.dk * d.r, torch.float32), _ptr(R, "R", d.H * d.r * d.dk, torch.float32),
         _ptr(workspace, "workspace"), ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+        ctypes.c_void_p(_stream(stream))))
+
+
+def sketchssm_calibrate_basis_noalloc(d: sketchssm_dims, q_cal, S_cal, U, R, ridge: float = 1e-8, stream=None):
+    """sketchssm_calibrate_basis for callers that cannot allocate device memory: the library
+    works in a fixed 3 MiB scratch array of its own (see include/sketchssm.h); neither the
+    library nor this wrapper allocates.  Calls that overlap on the GPU race on that scratch."""
+    Nq = q_cal.shape[1]
+    Ns = S_cal.shape[0]
+    _check("sketchssm_calibrate_basis_noalloc", library().sketchssm_calibrate_basis_noalloc(
+        ctypes.byref(d), _ptr(q_cal, "q_cal", d.H * Nq * d.dk, torch.float32), int(Nq),
+        _ptr(S_cal, "S_cal", Ns * d.H * d.dv * d.dk, _dt(d.state_dtype)), int(Ns), float(ridge),
+        _ptr(U, "U", d.H * d.dk * d.r, torch.float32), _ptr(R, "R", d.H * d.r * d.dk, torch.float32),
         ctypes.c_void_p(_stream(stream))))

@@ -300,4 +300,41 @@ int launch_calibrate(const sketchssm_dims &d, const float *q_cal, int Nq, const 
     return SKSSM_ERR_DIMS;
 }
 
+// Heads [h0, h0 + hc) only, with a workspace sized for hc heads: the same three
+// kernels as launch_calibrate, with every head-indexed pointer offset to h0.
+int launch_calibrate_heads(const sketchssm_dims &d, const float *q_cal, int Nq, const void *S_cal,
+                           int Ns, double ridge, float *U, float *R, void *workspace, int h0, int hc,
+                           cudaStream_t stream) {
+    double *G = static_cast<double *>(workspace);
+    double *C = G + (size_t)hc * d.dk * d.dk;
+    double *T = C + (size_t)hc * d.dk * d.dk;
+    auto run = [&](auto DKc) -> int {
+        constexpr int DK = decltype(DKc)::value;
+        const dim3 ggrid((DK / 32) * (DK / 32), hc);
+        const size_t sh = (size_t)d.dv * DK, sb = (size_t)d.H * d.dv * DK;
+        const size_t s_off = (size_t)h0 * d.dv * DK;
+        if (d.state_dtype == SKSSM_F32)
+            gram_kernel<float, DK><<<ggrid, 256, 0, stream>>>(static_cast<const float *>(S_cal) + s_off, sh,
+                                                              sb, d.dv, Ns * d.dv, 1.0 / Ns, G);
+        else
+            gram_kernel<__nv_bfloat16, DK><<<ggrid, 256, 0, stream>>>(
+                static_cast<const __nv_bfloat16 *>(S_cal) + s_off, sh, sb, d.dv, Ns * d.dv, 1.0 / Ns, G);
+        if (launch_status() != SKSSM_OK) return SKSSM_ERR_CUDA;
+        gram_kernel<float, DK><<<ggrid, 256, 0, stream>>>(q_cal + (size_t)h0 * Nq * DK, (size_t)Nq * DK, 0,
+                                                          Nq, Nq, 1.0 / Nq, C);
+        if (launch_status() != SKSSM_OK) return SKSSM_ERR_CUDA;
+        const size_t smem = basis_smem<DK>();
+        if (cudaFuncSetAttribute(basis_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem) != cudaSuccess)
+            return SKSSM_ERR_CUDA;
+        basis_kernel<DK><<<hc, BASIS_THREADS, smem, stream>>>(G, C, T, d.r, ridge,
+                                                               U + (size_t)h0 * DK * d.r,
+                                                               R + (size_t)h0 * d.r * DK);
+        return launch_status();
+    };
+    if (d.dk == 64) return run(std::integral_constant<int, 64>());
+    if (d.dk == 128) return run(std::integral_constant<int, 128>());
+    return SKSSM_ERR_DIMS;
+}
+
 }  // namespace skssm

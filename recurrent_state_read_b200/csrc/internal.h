@@ -54,5 +54,8 @@ int launch_decode_step(const sketchssm_dims &d, const float *P, const float *R, 
 size_t calibrate_workspace_bytes(const sketchssm_dims &d, int Nq, int Ns);
 int launch_calibrate(const sketchssm_dims &d, const float *q_cal, int Nq, const void *S_cal, int Ns,
                      double ridge, float *U, float *R, void *workspace, cudaStream_t stream);
+int launch_calibrate_heads(const sketchssm_dims &d, const float *q_cal, int Nq, const void *S_cal,
+                           int Ns, double ridge, float *U, float *R, void *workspace, int h0, int hc,
+                           cudaStream_t stream);
 
 }  // namespace skssm

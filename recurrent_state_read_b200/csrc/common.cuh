@@ -54,6 +54,19 @@ __device__ __forceinline__ void load16_stream<__nv_bfloat16>(const __nv_bfloat16
     out[4] = bf16lo(a.z); out[5] = bf16hi(a.z); out[6] = bf16lo(a.w); out[7] = bf16hi(a.w);
 }
 
+// Unpack one 16-byte vector of T to fp32.
+template <typename T>
+__device__ __forceinline__ void unpack16(const typename Vec<T>::type &a, float *out);
+template <>
+__device__ __forceinline__ void unpack16<float>(const float4 &a, float *out) {
+    out[0] = a.x; out[1] = a.y; out[2] = a.z; out[3] = a.w;
+}
+template <>
+__device__ __forceinline__ void unpack16<__nv_bfloat16>(const uint4 &a, float *out) {
+    out[0] = bf16lo(a.x); out[1] = bf16hi(a.x); out[2] = bf16lo(a.y); out[3] = bf16hi(a.y);
+    out[4] = bf16lo(a.z); out[5] = bf16hi(a.z); out[6] = bf16lo(a.w); out[7] = bf16hi(a.w);
+}
+
 // fp32 -> bf16 bits, round to nearest even (finite inputs; NaN kept quiet).
 __device__ __forceinline__ uint32_t bf16_bits(float x) {
     uint32_t u = __float_as_uint(x);

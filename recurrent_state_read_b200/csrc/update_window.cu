@@ -24,6 +24,70 @@
 
 namespace skssm {
 
+// Rows [0, n) of a strided token array (row t at src + t*row_stride + off, `len`
+// elements of T each) into fp32 shared memory dst[t*len + i].  Each thread
+// issues up to four 16-byte loads before converting any of them.
+template <typename T>
+__device__ __forceinline__ void stage_rows(const T *__restrict__ src, size_t row_stride, size_t off, int len,
+                                           int n, float *__restrict__ dst, int tid, int nthr) {
+    constexpr int V = Vec<T>::N;
+    const int per_row = len / V, total = n * per_row;
+    for (int base = tid; base < total; base += 4 * nthr) {
+        typename Vec<T>::type raw[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int idx = base + u * nthr;
+            if (idx < total) {
+                const int t = idx / per_row, c = (idx - t * per_row) * V;
+                raw[u] = *reinterpret_cast<const typename Vec<T>::type *>(src + (size_t)t * row_stride + off + c);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int idx = base + u * nthr;
+            if (idx < total) {
+                const int t = idx / per_row, c = (idx - t * per_row) * V;
+                float f[V];
+                unpack16<T>(raw[u], f);
+#pragma unroll
+                for (int e = 0; e < V; e += 4)
+                    *reinterpret_cast<float4 *>(dst + t * len + c + e) = make_float4(f[e], f[e + 1], f[e + 2], f[e + 3]);
+            }
+        }
+    }
+}
+
+// U [DK][r] (global, fp32) -> U^T [r][DK] in shared memory.
+__device__ __forceinline__ void stage_transposed(const float *__restrict__ Uh, int DK, int r,
+                                                 float *__restrict__ sut, int tid, int nthr) {
+    if ((r & 3) == 0) {
+        const int r4 = r / 4, total = DK * r4;
+        for (int idx = tid; idx < total; idx += nthr) {
+            const int i = idx / r4, m = (idx - i * r4) * 4;
+            const float4 a = *reinterpret_cast<const float4 *>(Uh + (size_t)i * r + m);
+            sut[(m + 0) * DK + i] = a.x;
+            sut[(m + 1) * DK + i] = a.y;
+            sut[(m + 2) * DK + i] = a.z;
+            sut[(m + 3) * DK + i] = a.w;
+        }
+    } else {
+        for (int idx = tid; idx < DK * r; idx += nthr) {
+            const int i = idx / r, m = idx - i * r;
+            sut[m * DK + i] = Uh[idx];
+        }
+    }
+}
+
+// Inclusive prefix product across the warp.
+__device__ __forceinline__ float warp_prefix_product(float x, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(FULL, x, o);
+        if (lane >= o) x *= y;
+    }
+    return x;
+}
+
 template <int KIND, int DK, typename ST, typename QT>
 __global__ void __launch_bounds__(128)
 update_window_kernel(ST *__restrict__ S, float *__restrict__ P, const float *__restrict__ U,
@@ -57,50 +121,46 @@ update_window_kernel(ST *__restrict__ S, float *__restrict__ P, const float *__r
     const ST *Sh = S + (size_t)head * dv * DK;
     load_tile<DK, ST>(Sh, c0, l, s);
 
-    // 2. stage the buffered tokens and U^T in shared memory
-    for (int idx = tid; idx < n * DK; idx += nthr) {
-        const int t = idx / DK, i = idx - t * DK;
-        sk[idx] = ld1(kbuf + ((size_t)t * NH + head) * DK + i);
-    }
-    for (int idx = tid; idx < n * dv; idx += nthr) {
-        const int t = idx / dv, c = idx - t * dv;
-        sv[idx] = ld1(vbuf + ((size_t)t * NH + head) * dv + c);
-    }
-    for (int idx = tid; idx < r * DK; idx += nthr) {
-        const int m = idx / DK, i = idx - m * DK;
-        sut[idx] = U[((size_t)h * DK + i) * r + m];
-    }
-    if (KIND != KDA) {
-        for (int t = tid; t < n; t += nthr) {
-            ss1[t] = abuf[(size_t)t * NH + head];
-            ss2[t] = KIND == GDN ? bbuf[(size_t)t * NH + head] : 1.f;
+    // 2. stage the buffered tokens and U^T in shared memory: every thread issues
+    //    all of its 16-byte loads before it converts and stores any of them
+    stage_rows<QT>(kbuf, (size_t)NH * DK, (size_t)head * DK, DK, n, sk, tid, nthr);
+    stage_rows<QT>(vbuf, (size_t)NH * dv, (size_t)head * dv, dv, n, sv, tid, nthr);
+    if (KIND == KDA) stage_rows<float>(abuf, (size_t)NH * DK, (size_t)head * DK, DK, n, sku, tid, nthr);
+    stage_transposed(U + (size_t)h * DK * r, DK, r, sut, tid, nthr);
+    if (KIND != KDA && warp == 0) {
+        // g_t = a_1 ... a_t by a warp prefix product (n <= 64: two tokens per lane)
+        float a0 = 1.f, a1 = 1.f, b0 = 1.f, b1 = 1.f;
+        if (lane < n) { a0 = abuf[(size_t)lane * NH + head]; if (KIND == GDN) b0 = bbuf[(size_t)lane * NH + head]; }
+        if (lane + 32 < n) {
+            a1 = abuf[(size_t)(lane + 32) * NH + head];
+            if (KIND == GDN) b1 = bbuf[(size_t)(lane + 32) * NH + head];
         }
+        const float p0 = warp_prefix_product(a0, lane);
+        const float p1 = warp_prefix_product(a1, lane) * __shfl_sync(FULL, p0, 31);
+        if (lane < n) { ss1[lane] = b0 / p0; ss2[lane] = b0; }
+        if (lane + 32 < n) { ss1[lane + 32] = b1 / p1; ss2[lane + 32] = b1; }
+        const float g_lo = __shfl_sync(FULL, p0, (n >= 1 && n <= 32) ? n - 1 : 31);
+        const float g_hi = __shfl_sync(FULL, p1, n > 32 ? n - 33 : 0);
+        if (lane == 0) sg[0] = n == 0 ? 1.f : (n <= 32 ? g_lo : g_hi);
     }
+    if (KIND == KDA)
+        for (int t = tid; t < n; t += nthr) ss2[t] = bbuf[(size_t)t * NH + head];
     __syncthreads();
-    if (KIND != KDA) {
-        if (tid == 0) {
-            float gam = 1.f;
-            for (int t = 0; t < n; ++t) {
-                gam *= ss1[t];
-                const float b = ss2[t];
-                ss1[t] = b / gam;  // Mamba-2: 1 / g_t;  GDN: b_t / g_t
-            }
-            sg[0] = gam;
-        }
-    } else {
+    if (KIND == KDA) {
+        // per key channel: g_{t,i} = a_{1,i} ... a_{t,i}; dot vector k g_t, update vector b k / g_t
         for (int i = tid; i < DK; i += nthr) {
             float gam = 1.f;
             for (int t = 0; t < n; ++t) {
-                gam *= abuf[((size_t)t * NH + head) * DK + i];
-                const float b = bbuf[(size_t)t * NH + head];
+                gam *= sku[t * DK + i];
+                const float b = ss2[t];
                 const float kr = sk[t * DK + i];
                 sk[t * DK + i] = kr * gam;
-                sku[t * DK + i] = b * kr / gam;
+                sku[t * DK + i] = b * kr * (1.f / gam);
             }
             sg[i] = gam;
         }
+        __syncthreads();
     }
-    __syncthreads();
 
     // 3. the buffered tokens, in order
     for (int t = 0; t < n; ++t) {
@@ -145,24 +205,31 @@ update_window_kernel(ST *__restrict__ S, float *__restrict__ P, const float *__r
     }
     if (n > 0) store_tile<DK, ST>(S + (size_t)head * dv * DK, c0, l, s);
 
-    // 5. sketch refresh P[c][m] = sum_i S[i][c] U[i][m], from the stored values
-    float *Ph = P + (size_t)head * dv * r;
+    // 5. sketch refresh P[c][m] = sum_i S[i][c] U[i][m], from the stored values: for
+    //    each m one dot per column and one reduce-scatter over the octet, after which
+    //    lane l holds P[c0 + l][m]
+    float *Prow = P + ((size_t)head * dv + c0 + l) * r;
     for (int m0 = 0; m0 < r; m0 += 8) {
+        float pm[8];
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-            float acc[8];
+        for (int mm = 0; mm < 8; ++mm) {
+            pm[mm] = 0.f;
+            if (m0 + mm < r) {
+                float uv[EPL];
+                lane_channels_smem<DK, ST>(sut + (m0 + mm) * DK, l, uv);
+                float d[8];
 #pragma unroll
-            for (int mm = 0; mm < 8; ++mm) {
-                if (m0 + mm < r) {
-                    float uv[EPL];
-                    lane_channels_smem<DK, ST>(sut + (m0 + mm) * DK, l, uv);
-                    acc[mm] = dot<EPL>(uv, s[cc]);
-                } else {
-                    acc[mm] = 0.f;
-                }
+                for (int cc = 0; cc < 8; ++cc) d[cc] = dot<EPL>(uv, s[cc]);
+                pm[mm] = octet_reduce_scatter(d, lane);
             }
-            const float pm = octet_reduce_scatter(acc, lane);
-            if (m0 + l < r) Ph[(size_t)(c0 + cc) * r + m0 + l] = pm;
+        }
+        if ((r & 3) == 0) {
+            *reinterpret_cast<float4 *>(Prow + m0) = make_float4(pm[0], pm[1], pm[2], pm[3]);
+            if (m0 + 4 < r) *reinterpret_cast<float4 *>(Prow + m0 + 4) = make_float4(pm[4], pm[5], pm[6], pm[7]);
+        } else {
+#pragma unroll
+            for (int mm = 0; mm < 8; ++mm)
+                if (m0 + mm < r) Prow[m0 + mm] = pm[mm];
         }
     }
 }

@@ -305,7 +305,7 @@ def run_ours(args):
     # start state: prefill through the library's window update
     S0 = torch.zeros(cfg.B, cfg.H, cfg.dv, cfg.dk, dtype=cfg.torch_state_dtype, device=dev)
     P = torch.empty(cfg.B, cfg.H, cfg.dv, cfg.r, device=dev)
-    U0 = torch.zeros(cfg.H, cfg.dk, cfg.r, device=dev)
+    U0 = torch.zeros(cfg.H, cfg.r, cfg.dk, device=dev)
     prefill(d, S0, P, U0, lambda t0, n: wl.token_block(cfg, "prefill", t0, n, device=dev), cfg.prefill)
     # offline basis: the library's calibration on prefilled calibration sequences
     dc = rs.dims(cfg.kind, cfg.n_cal_seq, cfg.H, cfg.dk, cfg.dv, cfg.r, cfg.W, cfg.torch_state_dtype,
@@ -314,17 +314,20 @@ def run_ours(args):
     P_cal = torch.empty(cfg.n_cal_seq, cfg.H, cfg.dv, cfg.r, device=dev)
     prefill(dc, S_cal, P_cal, U0, lambda t0, n: wl.token_block(cfg, "cal", t0, n, device=dev), cfg.prefill)
     q_cal = wl.calibration_queries(cfg, device=dev)
-    U = torch.empty(cfg.H, cfg.dk, cfg.r, device=dev)
+    U = torch.empty(cfg.H, cfg.r, cfg.dk, device=dev)  # basis rows
     R = torch.empty(cfg.H, cfg.r, cfg.dk, device=dev)
     rs.sketchssm_calibrate_basis(dc, q_cal, S_cal, U, R)
     del S_cal, P_cal, q_cal
 
     # NWIN distinct windows of decode tokens
-    bufs = []
+    bufs, toks = [], []
     for i in range(NWIN):
+        tok = wl.token_block(cfg, "decode", i * cfg.W, cfg.W, device=dev, with_query=True)  # time-major
+        tok = {k: (None if v is None else v.contiguous()) for k, v in tok.items()}
         b = WindowBuffer.empty(d, device=dev)
-        b.fill(wl.token_block(cfg, "decode", i * cfg.W, cfg.W, device=dev, with_query=True))
+        b.fill(tok)
         bufs.append(b)
+        toks.append(tok)  # the full-read baseline reads one token plane per step
     out = torch.empty(cfg.W, cfg.B, cfg.H, cfg.dv, device=dev)
     out_f = torch.empty_like(out)
     S = S0.clone()
@@ -337,7 +340,7 @@ def run_ours(args):
 
     S_a, Sf_a, P_a = S.clone(), S.clone(), P.clone()
     sketch_window(d, S_a, P_a, U, R, bufs[0], out)
-    fullread_window(d, Sf_a, bufs[0], out_f)
+    fullread_window(d, Sf_a, toks[0], out_f)
     torch.cuda.synchronize()
     approx = float(torch.linalg.vector_norm((out - out_f).double()) / torch.linalg.vector_norm(out_f.double()))
     del S_a, Sf_a, P_a
@@ -358,12 +361,12 @@ def run_ours(args):
     def upd_fn(b):
         return lambda: rs.sketchssm_update_window(d, S, P, U, b.k, b.v, b.alpha, b.beta, cfg.W)
 
-    def full_fn(b):
-        return lambda: fullread_window(d, Sf, b, out_f)
+    def full_fn(tok):
+        return lambda: fullread_window(d, Sf, tok, out_f)
 
     g_dec = [capture(dec_fn(b)) for b in bufs]
     g_upd = [capture(upd_fn(b)) for b in bufs]
-    g_full = [capture(full_fn(b)) for b in bufs]
+    g_full = [capture(full_fn(tok)) for tok in toks]
 
     uuid = None
     try:

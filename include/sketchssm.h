@@ -36,13 +36,15 @@
  *       S      [B][H][dv][dk]  state, stored transposed: row c holds column c of
  *                              S, i.e. S_T[n][c][i] = S[i][c]; dtype state_dtype
  *       P      [B][H][dv][r]   fp32 sketch, P[n][c][m] = sum_i S[i][c] U[i][m]
- *       U      [H][dk][r]      fp32 basis (per head h, shared by all b)
+ *       U      [H][r][dk]      fp32 basis stored as rows: U_rows[h][m][i] = U[i][m]
+ *                              (the dk x r basis of head h, shared by all b)
  *       R      [H][r][dk]      fp32 coefficient map, c = R q~
- *       window buffer, time-major, slot t = token t of the window:
- *       k      [W][B][H][dk]   qkv_dtype
- *       v      [W][B][H][dv]   qkv_dtype
- *       alpha  [W][B][H]       fp32 decay (SKSSM_KDA: [W][B][H][dk]); 4-byte aligned
- *       beta   [W][B][H]       fp32 (ignored, may be NULL, for SKSSM_MAMBA2); 4-byte aligned
+ *       window buffer, head-major (a head's W slots are contiguous), slot t =
+ *       token t of the window:
+ *       k      [B][H][W][dk]   qkv_dtype
+ *       v      [B][H][W][dv]   qkv_dtype
+ *       alpha  [B][H][W]       fp32 decay (SKSSM_KDA: [B][H][W][dk]); 4-byte aligned
+ *       beta   [B][H][W]       fp32 (ignored, may be NULL, for SKSSM_MAMBA2); 4-byte aligned
  *       q      [B][H][dk]      qkv_dtype, the current step's query
  *       o      [B][H][dv]      fp32 output
  *   - Supported sizes: dk in {64, 128}; dv in {64, 128}; 1 <= r <= 32 or r == dk;
@@ -100,7 +102,7 @@ int sketchssm_version(void);
  * n_tokens = 0 is a sketch refresh only (S is read, not written).
  *   S        in/out [B][H][dv][dk] state_dtype
  *   P        out    [B][H][dv][r] fp32
- *   U        in     [H][dk][r] fp32
+ *   U        in     [H][r][dk] fp32 (basis rows)
  *   k, v, alpha, beta  in: window buffer slots 0..n_tokens-1 (NULL allowed when
  *            n_tokens == 0; beta NULL allowed for SKSSM_MAMBA2)
  * Errors: ERR_NULL, ERR_DIMS, ERR_DTYPE, ERR_RANGE (n_tokens < 0 or > W),
@@ -148,6 +150,16 @@ int sketchssm_fullread_decode(const sketchssm_dims *dims, void *S, const void *q
                               void *stream);
 
 /*
+ * sketchssm_device_error_count -- kernels never wait without bound: the decode
+ * step's wait for its bulk copies gives up after a fixed number of attempts,
+ * counts the give-up in a device-side counter and returns without writing its
+ * output.  This call synchronises the current device and returns that count
+ * (0 in normal operation; a negative sketchssm_status if a CUDA call fails);
+ * reset != 0 clears it.
+ */
+int sketchssm_device_error_count(int reset);
+
+/*
  * sketchssm_calibrate_workspace_bytes -- device workspace that
  * sketchssm_calibrate_basis needs for these sizes (0 if dims are invalid).
  */
@@ -168,7 +180,7 @@ size_t sketchssm_calibrate_workspace_bytes(const sketchssm_dims *dims, int Nq, i
  *   S_cal  in  [Ns][H][dv][dk] calibration states in the S layout, state_dtype,
  *              Ns >= 1 (the B field of dims is ignored here)
  *   ridge  >= 0, relative diagonal guard (1e-8 is a good default)
- *   U out [H][dk][r] fp32;  R out [H][r][dk] fp32
+ *   U out [H][r][dk] fp32 (basis rows);  R out [H][r][dk] fp32
  *   workspace: device scratch of at least
  *              sketchssm_calibrate_workspace_bytes(dims, Nq, Ns) bytes, 256-byte
  *              aligned, owned by the caller; contents on entry are ignored.

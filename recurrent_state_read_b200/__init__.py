@@ -8,8 +8,9 @@ CPU fallback, and calling any entry point without the built library raises.
 
 Layouts (N = B*H heads, see include/sketchssm.h):
     S [B,H,dv,dk]  (state, transposed storage)   P [B,H,dv,r] fp32
-    U [H,dk,r] fp32      R [H,r,dk] fp32
-    window buffer: k [W,B,H,dk], v [W,B,H,dv], alpha [W,B,H] (KDA [W,B,H,dk]), beta [W,B,H]
+    U [H,r,dk] fp32 (basis rows, U_rows[h,m,i] = U[i,m])      R [H,r,dk] fp32
+    window buffer (head-major): k [B,H,W,dk], v [B,H,W,dv], alpha [B,H,W] (KDA [B,H,W,dk]), beta [B,H,W]
+    one token (full-read step): q, k [B,H,dk], v [B,H,dv], alpha [B,H] (KDA [B,H,dk]), beta [B,H]
     q [B,H,dk], o [B,H,dv] fp32
 """
 
@@ -35,6 +36,7 @@ EXPORTS = (
     "sketchssm_calibrate_workspace_bytes",
     "sketchssm_calibrate_basis",
     "sketchssm_calibrate_basis_noalloc",
+    "sketchssm_device_error_count",
 )
 
 
@@ -78,6 +80,8 @@ def library() -> ctypes.CDLL:
         lib.sketchssm_calibrate_basis.argtypes = [D, P, i, P, i, ctypes.c_double, P, P, P,
                                                   ctypes.c_size_t, P]
         lib.sketchssm_calibrate_basis_noalloc.argtypes = [D, P, i, P, i, ctypes.c_double, P, P, P]
+        lib.sketchssm_device_error_count.argtypes = [i]
+        lib.sketchssm_device_error_count.restype = i
         for f in ("sketchssm_update_window", "sketchssm_decode_step", "sketchssm_fullread_decode",
                   "sketchssm_calibrate_basis", "sketchssm_calibrate_basis_noalloc"):
             getattr(lib, f).restype = i
@@ -121,13 +125,15 @@ def _check(fn: str, rc: int):
         raise SketchSSMError(fn, rc, library().sketchssm_status_string(rc).decode())
 
 
-def _token_ptrs(d: sketchssm_dims, n: int, k, v, alpha, beta):
+def _token_ptrs(d: sketchssm_dims, slots: int, k, v, alpha, beta):
+    """Pointers of `slots` tokens per head: slots = W for a head-major window buffer
+    [B,H,W,..], slots = 1 for the single token plane [B,H,..] of a full-read step."""
     NH = d.B * d.H
     qt = _dt(d.qkv_dtype)
     na = d.dk if d.kind == KIND["kda"] else 1
-    return (_ptr(k, "k", n * NH * d.dk, qt), _ptr(v, "v", n * NH * d.dv, qt),
-            _ptr(alpha, "alpha", n * NH * na, torch.float32),
-            _ptr(beta, "beta", n * NH, torch.float32))
+    return (_ptr(k, "k", slots * NH * d.dk, qt), _ptr(v, "v", slots * NH * d.dv, qt),
+            _ptr(alpha, "alpha", slots * NH * na, torch.float32),
+            _ptr(beta, "beta", slots * NH, torch.float32))
 
 
 def sketchssm_update_window(d: sketchssm_dims, S, P, U, k, v, alpha, beta, n_tokens: int, stream=None):
@@ -135,7 +141,7 @@ def sketchssm_update_window(d: sketchssm_dims, S, P, U, k, v, alpha, beta, n_tok
     NH = d.B * d.H
     args = (_ptr(S, "S", NH * d.dv * d.dk, _dt(d.state_dtype)), _ptr(P, "P", NH * d.dv * d.r, torch.float32),
             _ptr(U, "U", d.H * d.dk * d.r, torch.float32))
-    toks = _token_ptrs(d, n_tokens, k, v, alpha, beta) if n_tokens > 0 else (None,) * 4
+    toks = _token_ptrs(d, d.W, k, v, alpha, beta) if n_tokens > 0 else (None,) * 4
     _check("sketchssm_update_window",
            library().sketchssm_update_window(ctypes.byref(d), *args, *toks, int(n_tokens),
                                              ctypes.c_void_p(_stream(stream))))
@@ -144,7 +150,7 @@ def sketchssm_update_window(d: sketchssm_dims, S, P, U, k, v, alpha, beta, n_tok
 def sketchssm_decode_step(d: sketchssm_dims, P, R, q, k, v, alpha, beta, j: int, o, stream=None):
     """Decode step j of the window from the sketch P and window-buffer tokens 0..j-1 into o."""
     NH = d.B * d.H
-    toks = _token_ptrs(d, j, k, v, alpha, beta)
+    toks = _token_ptrs(d, d.W, k, v, alpha, beta)
     _check("sketchssm_decode_step", library().sketchssm_decode_step(
         ctypes.byref(d), _ptr(P, "P", NH * d.dv * d.r, torch.float32),
         _ptr(R, "R", d.H * d.r * d.dk, torch.float32), _ptr(q, "q", NH * d.dk, _dt(d.qkv_dtype)),
@@ -167,7 +173,7 @@ def sketchssm_calibrate_workspace_bytes(d: sketchssm_dims, Nq: int, Ns: int) -> 
 
 def sketchssm_calibrate_basis(d: sketchssm_dims, q_cal, S_cal, U, R, workspace=None, ridge: float = 1e-8,
                               stream=None):
-    """Offline basis: q_cal [H,Nq,dk] fp32, S_cal [Ns,H,dv,dk] -> U [H,dk,r], R [H,r,dk].
+    """Offline basis: q_cal [H,Nq,dk] fp32, S_cal [Ns,H,dv,dk] -> U [H,r,dk] (rows), R [H,r,dk].
 
     `workspace` is a uint8 CUDA tensor of at least sketchssm_calibrate_workspace_bytes bytes; when
     None, one is allocated here through torch (the library itself never allocates).
@@ -196,3 +202,11 @@ def sketchssm_calibrate_basis_noalloc(d: sketchssm_dims, q_cal, S_cal, U, R, rid
         _ptr(S_cal, "S_cal", Ns * d.H * d.dv * d.dk, _dt(d.state_dtype)), int(Ns), float(ridge),
         _ptr(U, "U", d.H * d.dk * d.r, torch.float32), _ptr(R, "R", d.H * d.r * d.dk, torch.float32),
         ctypes.c_void_p(_stream(stream))))
+
+
+def sketchssm_device_error_count(reset: bool = False) -> int:
+    """Bounded in-kernel waits that gave up on the current device (0 in normal operation)."""
+    n = int(library().sketchssm_device_error_count(int(reset)))
+    if n < 0:
+        raise SketchSSMError("sketchssm_device_error_count", n, library().sketchssm_status_string(n).decode())
+    return n

@@ -17,6 +17,7 @@
 //                 cyclic Jacobi with a round-robin pair ordering (dk/2 disjoint
 //                 rotations per round, at most 40 sweeps), top-r selection,
 //                 back substitution for U, and R = V_r^T L^T.
+// U is written as basis rows, U_rows[h][m][i] = U[i][m], like R.
 // Workspace (caller-owned): G/L, C, T/V, each [H][dk][dk] fp64.
 #include <math.h>
 
@@ -246,8 +247,8 @@ basis_kernel(double *__restrict__ Gw, const double *__restrict__ Cw, double *__r
     }
     __syncthreads();
     for (int idx = tid; idx < DK * r; idx += BASIS_THREADS) {
-        const int i = idx / r, m = idx % r;
-        U[((size_t)h * DK + i) * r + m] = (float)X[m * DK + i];
+        const int m = idx / DK, i = idx % DK;
+        U[((size_t)h * r + m) * DK + i] = (float)X[m * DK + i];
     }
     for (int idx = tid; idx < r * DK; idx += BASIS_THREADS) {
         const int m = idx / DK, i = idx % DK;

@@ -182,6 +182,29 @@ __device__ __forceinline__ void octet_all_gather(float x, float (&out)[8]) {
     for (int m = 0; m < 8; ++m) out[m] = __shfl_sync(FULL, x, m, 8);
 }
 
+// Octet reduction of 4 values: on entry lane l holds partials d[0..3]; on exit
+// lanes l and l^1 both hold the octet-wide sum of d[(l & 7) >> 1].  4 shuffles.
+__device__ __forceinline__ float octet_reduce4(const float (&d)[4], int lane) {
+    const bool b2 = lane & 4, b1 = lane & 2;
+    float a[2];
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+        float send = b2 ? d[m] : d[m + 2];
+        float keep = b2 ? d[m + 2] : d[m];
+        a[m] = keep + __shfl_xor_sync(FULL, send, 4);
+    }
+    float send = b1 ? a[0] : a[1];
+    float keep = b1 ? a[1] : a[0];
+    float x = keep + __shfl_xor_sync(FULL, send, 2);
+    return x + __shfl_xor_sync(FULL, x, 1);
+}
+
+// out[m] = value held by octet lanes 2m (and 2m+1) after octet_reduce4.
+__device__ __forceinline__ void octet_all_gather4(float x, float (&out)[4]) {
+#pragma unroll
+    for (int m = 0; m < 4; ++m) out[m] = __shfl_sync(FULL, x, 2 * m, 8);
+}
+
 __device__ __forceinline__ float octet_sum(float x) {
     x += __shfl_xor_sync(FULL, x, 1);
     x += __shfl_xor_sync(FULL, x, 2);

@@ -5,15 +5,16 @@
 // sketch refresh act on each column independently, and every reduction they
 // need (k . S[:,c], q . S[:,c], U^T S[:,c]) runs along that contiguous vector.
 //
-// A warp owns 32 columns.  Lane = 8 g + l holds the 8 columns c0 + cc
-// (c0 = 32 warp + 8 g, cc < 8) and, in each of them, the key channels
+// A warp owns 4 NC columns.  Lane = 8 g + l holds the NC columns c0 + cc
+// (c0 = 4 NC warp + NC g, cc < NC; NC = 8 or 4) and, in each of them, the key channels
 //     i = VEC (l + 8 q) + e,   q < NQ, e < VEC,
 // where VEC elements fill one 16-byte vector of the storage type.  One warp-wide
 // 16-byte load instruction therefore reads four 128-byte runs (one per lane
 // octet), every byte of which is used.  A column's reductions are a per-lane
 // partial over EPL = dk/8 channels followed by a reduction across the 8 lanes
-// of an octet; 8 columns per lane let one octet reduce-scatter (7 shuffles)
-// and all-gather (8 shuffles) serve 8 columns at a time.
+// of an octet; with 8 columns per lane one octet reduce-scatter (7 shuffles)
+// and all-gather (8 shuffles) serve 8 columns at a time, with 4 columns per
+// lane 4 + 4 shuffles serve 4 (and half the registers hold the tile).
 #pragma once
 
 #include "common.cuh"
@@ -55,21 +56,21 @@ __device__ __forceinline__ void lane_channels_global(const QT *x, int l, float (
         for (int e4 = 0; e4 < TL::VEC; e4 += 4) load4(x + TL::chan(l, q, e4), out + q * TL::VEC + e4);
 }
 
-template <int DK, typename ST>
-__device__ __forceinline__ void load_tile(const ST *Sh, int c0, int l, float (&s)[8][DK / 8]) {
+template <int DK, typename ST, int NC = 8>
+__device__ __forceinline__ void load_tile(const ST *Sh, int c0, int l, float (&s)[NC][DK / 8]) {
     using TL = TileLayout<DK, ST>;
 #pragma unroll
-    for (int cc = 0; cc < 8; ++cc)
+    for (int cc = 0; cc < NC; ++cc)
 #pragma unroll
         for (int q = 0; q < TL::NQ; ++q)
             load16_stream<ST>(Sh + (size_t)(c0 + cc) * DK + TL::chan(l, q, 0), &s[cc][q * TL::VEC]);
 }
 
-template <int DK, typename ST>
-__device__ __forceinline__ void store_tile(ST *Sh, int c0, int l, const float (&s)[8][DK / 8]) {
+template <int DK, typename ST, int NC = 8>
+__device__ __forceinline__ void store_tile(ST *Sh, int c0, int l, const float (&s)[NC][DK / 8]) {
     using TL = TileLayout<DK, ST>;
 #pragma unroll
-    for (int cc = 0; cc < 8; ++cc)
+    for (int cc = 0; cc < NC; ++cc)
 #pragma unroll
         for (int q = 0; q < TL::NQ; ++q)
             store16_stream<ST>(Sh + (size_t)(c0 + cc) * DK + TL::chan(l, q, 0), &s[cc][q * TL::VEC]);

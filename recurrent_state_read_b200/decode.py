@@ -21,8 +21,9 @@ from . import (sketchssm_decode_step, sketchssm_dims, sketchssm_fullread_decode,
 
 @dataclasses.dataclass
 class WindowBuffer:
-    """Device window buffer, time-major: k [W,B,H,dk], v [W,B,H,dv], alpha [W,B,H(,dk)],
-    beta [W,B,H] (None for Mamba-2), q [W,B,H,dk] (the queries of the window's steps)."""
+    """Device window buffer, head-major: k [B,H,W,dk], v [B,H,W,dv], alpha [B,H,W] (KDA
+    [B,H,W,dk]), beta [B,H,W] (None for Mamba-2); q [W,B,H,dk] holds the queries of the
+    window's steps (one [B,H,dk] plane per step)."""
     k: torch.Tensor
     v: torch.Tensor
     alpha: torch.Tensor
@@ -33,22 +34,25 @@ class WindowBuffer:
     def empty(d: sketchssm_dims, device="cuda", with_query=True) -> "WindowBuffer":
         qt = torch.float32 if d.qkv_dtype == 0 else torch.bfloat16
         W, B, H = d.W, d.B, d.H
-        a_shape = (W, B, H, d.dk) if d.kind == 2 else (W, B, H)
+        a_shape = (B, H, W, d.dk) if d.kind == 2 else (B, H, W)
         return WindowBuffer(
-            k=torch.empty(W, B, H, d.dk, dtype=qt, device=device),
-            v=torch.empty(W, B, H, d.dv, dtype=qt, device=device),
+            k=torch.empty(B, H, W, d.dk, dtype=qt, device=device),
+            v=torch.empty(B, H, W, d.dv, dtype=qt, device=device),
             alpha=torch.empty(a_shape, dtype=torch.float32, device=device),
-            beta=None if d.kind == 0 else torch.empty(W, B, H, dtype=torch.float32, device=device),
+            beta=None if d.kind == 0 else torch.empty(B, H, W, dtype=torch.float32, device=device),
             q=torch.empty(W, B, H, d.dk, dtype=qt, device=device) if with_query else None,
         )
 
     def fill(self, tok: dict, n: Optional[int] = None):
-        """Copy tokens (dict of [n,B,H,...] tensors) into slots 0..n-1."""
+        """Copy time-major tokens (dict of [n,B,H,...] tensors) into slots 0..n-1."""
         n = tok["k"].shape[0] if n is None else n
-        for name in ("k", "v", "alpha", "beta", "q"):
+        for name in ("k", "v", "alpha", "beta"):
             dst = getattr(self, name)
             if dst is not None and tok.get(name) is not None:
-                dst[:n].copy_(tok[name][:n], non_blocking=True)
+                src = tok[name][:n]
+                dst[:, :, :n].copy_(src.movedim(0, 2), non_blocking=True)
+        if self.q is not None and tok.get("q") is not None:
+            self.q[:n].copy_(tok["q"][:n], non_blocking=True)
 
 
 def sketch_window(d: sketchssm_dims, S, P, U, R, buf: WindowBuffer, out, n: Optional[int] = None,
@@ -62,19 +66,21 @@ def sketch_window(d: sketchssm_dims, S, P, U, R, buf: WindowBuffer, out, n: Opti
     sketchssm_update_window(d, S, P, U, buf.k, buf.v, buf.alpha, buf.beta, n, stream)
 
 
-def fullread_window(d: sketchssm_dims, S, buf: WindowBuffer, out, n: Optional[int] = None, stream=None):
-    """n steps of the full-read baseline over the same window buffer."""
-    n = d.W if n is None else n
+def fullread_window(d: sketchssm_dims, S, tok: dict, out, n: Optional[int] = None, stream=None):
+    """n steps of the full-read baseline over time-major tokens (dict of contiguous
+    [n,B,H,...] device tensors k, v, alpha, beta, q): one token plane per step."""
+    n = tok["k"].shape[0] if n is None else n
+    beta = tok.get("beta")
     for t in range(n):
-        sketchssm_fullread_decode(d, S, buf.q[t], buf.k[t], buf.v[t], buf.alpha[t],
-                                  None if buf.beta is None else buf.beta[t], out[t], stream)
+        sketchssm_fullread_decode(d, S, tok["q"][t], tok["k"][t], tok["v"][t], tok["alpha"][t],
+                                  None if beta is None else beta[t], out[t], stream)
 
 
 def prefill(d: sketchssm_dims, S, P, U, token_source, n_tokens: int, stream=None):
     """Advance S through n_tokens tokens with window updates of up to W tokens each.
 
-    token_source(t0, n) returns a dict of device tensors [n,B,H,...] for tokens t0..t0+n-1.
-    P is refreshed as a by-product (the last refresh is the sketch of the final state).
+    token_source(t0, n) returns a dict of time-major device tensors [n,B,H,...] for tokens
+    t0..t0+n-1.  P is refreshed as a by-product (the last refresh is the sketch of the final state).
     """
     buf = WindowBuffer.empty(d, device=S.device, with_query=False)
     for t0 in range(0, n_tokens, d.W):

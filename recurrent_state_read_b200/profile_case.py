@@ -46,10 +46,11 @@ def main():
     g = torch.Generator(device=dev).manual_seed(0)
     S = (0.1 * torch.randn(cfg.B, cfg.H, cfg.dv, cfg.dk, generator=g, device=dev)).to(cfg.torch_state_dtype)
     P = torch.randn(cfg.B, cfg.H, cfg.dv, cfg.r, generator=g, device=dev)
-    U = torch.randn(cfg.H, cfg.dk, cfg.r, generator=g, device=dev) / cfg.dk ** 0.5
+    U = torch.randn(cfg.H, cfg.r, cfg.dk, generator=g, device=dev) / cfg.dk ** 0.5  # basis rows
     R = torch.randn(cfg.H, cfg.r, cfg.dk, generator=g, device=dev) / cfg.dk ** 0.5
+    tok = wl.token_block(cfg, "decode", 0, cfg.W, device=dev, with_query=True)  # time-major
     buf = WindowBuffer.empty(d, device=dev)
-    buf.fill(wl.token_block(cfg, "decode", 0, cfg.W, device=dev, with_query=True))
+    buf.fill(tok)
     o = torch.empty(cfg.B, cfg.H, cfg.dv, device=dev)
     j = cfg.W if a.j is None else a.j
 
@@ -59,8 +60,8 @@ def main():
         elif a.kernel == "decode":
             rs.sketchssm_decode_step(d, P, R, buf.q[j - 1], buf.k, buf.v, buf.alpha, buf.beta, j, o)
         else:
-            rs.sketchssm_fullread_decode(d, S, buf.q[0], buf.k[0], buf.v[0], buf.alpha[0],
-                                         None if buf.beta is None else buf.beta[0], o)
+            rs.sketchssm_fullread_decode(d, S, tok["q"][0], tok["k"][0], tok["v"][0], tok["alpha"][0],
+                                         None if tok["beta"] is None else tok["beta"][0], o)
 
     launch()
     torch.cuda.synchronize()

@@ -69,3 +69,8 @@ def rel_l2(a, b) -> float:
 
 def to_device(tok: dict, device="cuda") -> dict:
     return {k: (None if v is None else v.to(device).contiguous()) for k, v in tok.items()}
+
+
+def to_window(tok: dict) -> dict:
+    """Time-major tokens [W,B,H,...] -> the head-major window buffer layout [B,H,W,...]."""
+    return {k: (None if v is None else v.movedim(0, 2).contiguous()) for k, v in tok.items()}

@@ -44,11 +44,11 @@ def test_calibrate_matches_oracle(cid, n_seq, n_tokens, n_q, r):
     U_ref, R_ref = oracle.calibrate_heads(S_cal, q_cal.double().numpy(), r)
     d = rs.dims(cfg.kind, n_seq, cfg.H, cfg.dk, cfg.dv, r, cfg.W, torch.float32, cfg.torch_qkv_dtype)
     S_gpu = to_gpu_state(S_cal.reshape(n_seq * cfg.H, cfg.dk, cfg.dv), n_seq, cfg.H)
-    U = torch.full((cfg.H, cfg.dk, r), float("nan"), device="cuda")
+    U = torch.full((cfg.H, r, cfg.dk), float("nan"), device="cuda")  # basis rows
     R = torch.full((cfg.H, r, cfg.dk), float("nan"), device="cuda")
     rs.sketchssm_calibrate_basis(d, q_cal.cuda().contiguous(), S_gpu, U, R)
     torch.cuda.synchronize()
-    U, R = U.double().cpu().numpy(), R.double().cpu().numpy()
+    U, R = U.transpose(1, 2).double().cpu().numpy(), R.double().cpu().numpy()
     for h in range(cfg.H):
         Pi, Pi_ref = U[h] @ R[h], U_ref[h] @ R_ref[h]
         scale = max(1.0, np.abs(Pi_ref).max())
@@ -69,11 +69,11 @@ def test_calibrate_bf16_states():
     U_ref, R_ref = oracle.calibrate_heads(S_cal, q_cal.double().numpy(), 8)
     d = rs.dims("gdn", 16, cfg.H, 128, 128, 8, 16, torch.bfloat16, torch.bfloat16)
     S_gpu = to_gpu_state(S_cal.reshape(-1, 128, 128), 16, cfg.H, torch.bfloat16)
-    U = torch.empty(cfg.H, 128, 8, device="cuda")
+    U = torch.empty(cfg.H, 8, 128, device="cuda")  # basis rows
     R = torch.empty(cfg.H, 8, 128, device="cuda")
     rs.sketchssm_calibrate_basis(d, q_cal.cuda().contiguous(), S_gpu, U, R)
     torch.cuda.synchronize()
     for h in range(cfg.H):
-        Pi = U[h].double().cpu().numpy() @ R[h].double().cpu().numpy()
+        Pi = U[h].T.double().cpu().numpy() @ R[h].double().cpu().numpy()
         Pi_ref = U_ref[h] @ R_ref[h]
         assert np.abs(Pi - Pi_ref).max() <= 1e-5 * max(1.0, np.abs(Pi_ref).max())

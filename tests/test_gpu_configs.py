@@ -57,16 +57,17 @@ def _run_gpu(cfg, S0_gpu, U, R, source, n_steps):
     S = S0_gpu.clone()
     Sf = S0_gpu.clone()
     P = torch.empty(cfg.B, cfg.H, cfg.dv, cfg.r, device="cuda")
-    Ug, Rg = U.float().cuda().contiguous(), R.float().cuda().contiguous()
+    Ug, Rg = U.float().transpose(1, 2).contiguous().cuda(), R.float().cuda().contiguous()  # U as rows
     rs.sketchssm_update_window(d, S, P, Ug, None, None, None, None, 0)
     buf = WindowBuffer.empty(d)
     o_s = torch.empty(n_steps, cfg.B, cfg.H, cfg.dv, device="cuda")
     o_f = torch.empty_like(o_s)
     for t0 in range(0, n_steps, cfg.W):
         n = min(cfg.W, n_steps - t0)
-        buf.fill(source(t0, n), n)
+        tok = {k: (None if v is None else v.contiguous()) for k, v in source(t0, n).items()}
+        buf.fill(tok, n)
         sketch_window(d, S, P, Ug, Rg, buf, o_s[t0:t0 + n], n)
-        fullread_window(d, Sf, buf, o_f[t0:t0 + n], n)
+        fullread_window(d, Sf, tok, o_f[t0:t0 + n], n)
     torch.cuda.synchronize()
     return o_s, o_f, S, Sf, P
 
@@ -125,7 +126,7 @@ def _sampled(cfg, n_windows=2, n_heads=48, cal=(8, 64, 512), label=""):
     # GPU prefill over all heads; the oracle prefills the sampled heads from the same tokens
     S0 = torch.zeros(cfg.B, cfg.H, cfg.dv, cfg.dk, dtype=cfg.torch_state_dtype, device="cuda")
     P = torch.empty(cfg.B, cfg.H, cfg.dv, cfg.r, device="cuda")
-    Uz = torch.zeros(cfg.H, cfg.dk, cfg.r, device="cuda")
+    Uz = torch.zeros(cfg.H, cfg.r, cfg.dk, device="cuda")
     sampled_pre = []
 
     def pre_source(t0, n):

@@ -16,7 +16,7 @@ import torch
 import oracle
 import workloads as wl
 from tests.helpers import (BF16_OUT_TOL, BF16_STATE_TOL, STATE_TOL, TIGHT_OUT, flat_tokens, rel_l2,
-                           state_err, to_device, to_gpu_state, to_logical)
+                           state_err, to_device, to_gpu_state, to_logical, to_window)
 
 pytestmark = pytest.mark.gpu
 
@@ -74,11 +74,12 @@ def test_update_window(case):
     heads = np.arange(B * H)
     Uh = oracle.per_head(U, H, heads)
     ft = flat_tokens(tok)
-    dev = to_device(tok)
+    dev = to_window(to_device(tok))
     for n in sorted({0, 1, max(1, W // 2), W}):
         S = to_gpu_state(S0, B, H, sdt)
         P = torch.full((B, H, dv, r), float("nan"), device="cuda")
-        rs.sketchssm_update_window(d, S, P, U.cuda(), dev["k"], dev["v"], dev["alpha"], dev["beta"], n)
+        rs.sketchssm_update_window(d, S, P, U.transpose(1, 2).contiguous().cuda(), dev["k"], dev["v"],
+                                   dev["alpha"], dev["beta"], n)
         torch.cuda.synchronize()
         sl = slice(0, n)
         Sref, Pref = oracle.update_window(kind, S0, Uh, ft["k"][sl] if n else None, ft["v"][sl],
@@ -105,11 +106,12 @@ def test_decode_step(case):
     P = torch.randn(B, H, dv, r, generator=g)
     ft = flat_tokens(tok)
     dev = to_device(tok)
+    win = to_window(dev)
     Rh = oracle.per_head(R, H, heads)
     for j in sorted({1, max(1, W // 2), W}):
         o = torch.full((B, H, dv), float("nan"), device="cuda")
-        rs.sketchssm_decode_step(d, P.cuda(), R.cuda(), dev["q"][j - 1], dev["k"], dev["v"], dev["alpha"],
-                                 dev["beta"], j, o)
+        rs.sketchssm_decode_step(d, P.cuda(), R.cuda(), dev["q"][j - 1], win["k"], win["v"], win["alpha"],
+                                 win["beta"], j, o)
         torch.cuda.synchronize()
         sl = slice(0, j)
         ref = oracle.sketch_read(kind, P.reshape(B * H, dv, r), Rh, ft["q"][j - 1], ft["k"][sl], ft["v"][sl],
@@ -152,6 +154,7 @@ def test_complete_basis_sketch_is_exact_read():
     B, H = d.B, d.H
     eye = torch.eye(dk).expand(H, dk, dk).contiguous().cuda()
     dev = to_device(tok)
+    win = to_window(dev)
     S = to_gpu_state(S0, B, H)
     Sf = S.clone()
     P = torch.empty(B, H, dv, dk, device="cuda")
@@ -159,7 +162,7 @@ def test_complete_basis_sketch_is_exact_read():
     o_s = torch.empty(W, B, H, dv, device="cuda")
     o_f = torch.empty(W, B, H, dv, device="cuda")
     for j in range(1, W + 1):
-        rs.sketchssm_decode_step(d, P, eye, dev["q"][j - 1], dev["k"], dev["v"], dev["alpha"], dev["beta"],
+        rs.sketchssm_decode_step(d, P, eye, dev["q"][j - 1], win["k"], win["v"], win["alpha"], win["beta"],
                                  j, o_s[j - 1])
         rs.sketchssm_fullread_decode(d, Sf, dev["q"][j - 1], dev["k"][j - 1], dev["v"][j - 1],
                                      dev["alpha"][j - 1], dev["beta"][j - 1], o_f[j - 1])
@@ -192,3 +195,10 @@ def test_invalid_arguments_launch_nothing():
     assert e.value.status == -3
     torch.cuda.synchronize()
     assert torch.count_nonzero(S) == 0 and torch.count_nonzero(P) == 0
+
+
+def test_no_bounded_wait_gave_up():
+    """Every bounded in-kernel wait in the runs above completed (none gave up)."""
+    import recurrent_state_read_b200 as rs
+
+    assert rs.sketchssm_device_error_count() == 0

@@ -25,18 +25,18 @@ def test_noalloc_matches_workspace_entry_point(kind, H, dk, dv, r):
     g = torch.Generator(device="cuda").manual_seed(5)
     S_cal = torch.randn(Ns, H, dv, dk, generator=g, device="cuda")
     d = rs.dims(kind, Ns, H, dk, dv, r, 16, torch.float32, torch.bfloat16)
-    U_ref = torch.empty(H, dk, r, device="cuda")
+    U_ref = torch.empty(H, r, dk, device="cuda")  # basis rows
     R_ref = torch.empty(H, r, dk, device="cuda")
     for call in range(2):
         q_cal = torch.randn(H, Nq, dk, generator=g, device="cuda")
         rs.sketchssm_calibrate_basis(d, q_cal, S_cal, U_ref, R_ref)
-        U = torch.full((H, dk, r), float("nan"), device="cuda")
+        U = torch.full((H, r, dk), float("nan"), device="cuda")
         R = torch.full((H, r, dk), float("nan"), device="cuda")
         rs.sketchssm_calibrate_basis_noalloc(d, q_cal, S_cal, U, R)
         torch.cuda.synchronize()
         assert torch.isfinite(U).all() and torch.isfinite(R).all(), call
-        Pi = torch.einsum("hir,hrk->hik", U.double(), R.double())
-        Pi_ref = torch.einsum("hir,hrk->hik", U_ref.double(), R_ref.double())
+        Pi = torch.einsum("hri,hrk->hik", U.double(), R.double())
+        Pi_ref = torch.einsum("hri,hrk->hik", U_ref.double(), R_ref.double())
         scale = max(1.0, float(Pi_ref.abs().max()))
         assert float((Pi - Pi_ref).abs().max()) <= 1e-5 * scale, call
         assert torch.allclose(U, U_ref, rtol=1e-5, atol=1e-6 * float(U_ref.abs().max())), call

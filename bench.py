@@ -279,6 +279,26 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- multi-rank plumbing
+def reduce_max(x: float, device=None) -> float:
+    """Max of x over all ranks (identity without an initialised process group).
+
+    With NCCL the value travels in a CUDA tensor on `device`; with gloo on the CPU."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, t_max: float) -> float:
+    """Replicas: every rank processes the same units; the job's rate is all units over the slowest rank."""
+    return world * units_per_rank / t_max
+
+
 # ---------------------------------------------------------------- GPU arm
 def run_ours(args):
     import torch
@@ -382,11 +402,7 @@ def run_ours(args):
         torch.cuda.synchronize()
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, dev)
 
     def ev():
         return torch.cuda.Event(enable_timing=True)
@@ -456,15 +472,15 @@ def run_ours(args):
         barrier()
         clocks.mark(False)
         t_e2e = max_over_ranks(ee0.elapsed_time(ee1) / 1e3)
-        e2e = {"value": world * args.steps * cfg.B * cfg.W / t_e2e, "unit": UNIT,
+        e2e = {"value": whole_job_rate(args.steps * cfg.B * cfg.W, world, t_e2e), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": 1e3 * t_e2e / args.steps,
                "path": "python binding -> C ABI; pinned-host window inputs copied in and outputs copied "
                        "out every step, inside the timed region"}
     clk = clocks.stop()
 
     tok_per_step = cfg.B * cfg.W
-    value = world * args.steps * tok_per_step / t_sketch
-    value_full = world * args.steps * tok_per_step / t_full
+    value = whole_job_rate(args.steps * tok_per_step, world, t_sketch)
+    value_full = whole_job_rate(args.steps * tok_per_step, world, t_full)
     peak, peak_src = hbm_peak()
     upd_ms = 1e3 * t_upd / args.steps
     dec_ms = 1e3 * t_dec / (args.steps * cfg.W)

@@ -5,14 +5,14 @@
 // into a compact sketch; agihunt digest, bullet "Error control": the window's
 // state update and the sketch refresh happen in the same kernel.
 //
-// One CTA per head (b, h), dv/16 warps, each warp owning 16 value columns of S
-// (state_tile.cuh layout, 4 columns per lane).  The CTA loads the head's state
+// One CTA per head (b, h), dv/32 warps, each warp owning 32 value columns of S
+// (state_tile.cuh layout, 8 columns per lane).  The CTA loads the head's state
 // straight into registers with 16-byte streaming loads, stages the window's
 // tokens once in shared memory (converted to fp32, per-token scalars folded
 // in), applies the n tokens in order from registers, stores the state once and
-// writes P = S^T U from the same registers.  The register tile is kept small
-// (64 values per lane) so that several CTAs share an SM: while one applies its
-// tokens, the others' state loads are in flight.
+// writes P = S^T U from the same registers (basis rows staged in shared memory).
+// Several CTAs share an SM: while one applies its tokens, the others' state
+// loads are in flight.
 //
 // Scalar decay (Mamba-2, GDN) is folded into a running scale: S_t = g_t S^_t
 // with g_t = a_1 ... a_t, so a token costs one dot product and one rank-1
@@ -27,7 +27,7 @@
 
 namespace skssm {
 
-constexpr int UPD_NC = 4;  // value columns per lane (state_tile.cuh)
+constexpr int UPD_NC = 8;  // value columns per lane (state_tile.cuh)
 
 // Inclusive prefix product across the warp.
 __device__ __forceinline__ float warp_prefix_product(float x, int lane) {
@@ -100,14 +100,19 @@ update_window_kernel(ST *__restrict__ S, float *__restrict__ P, const float *__r
     float *su = sk + (size_t)n * DK;                       // [n][DK] (KDA)
     float *sv = su + (KIND == KDA ? (size_t)n * DK : 0);   // [n][dv]
     float *sg = sv + (size_t)n * dv;                       // [DK]
-    float *ss1 = sg + DK;                                  // [n4]: b_t / g_t (Mamba-2: 1 / g_t)
+    float *sut = sg + DK;                                  // [r][DK]: the head's basis rows
+    float *ss1 = sut + (size_t)r * DK;                     // [n4]: b_t / g_t (Mamba-2: 1 / g_t)
     float *ss2 = ss1 + ((n + 3) & ~3);                     // [n4]: b_t
 
     // 1. the state goes in flight first, straight into registers
     float s[NC][EPL];
     load_tile<DK, ST, NC>(S + (size_t)head * dv * DK, c0, l, s);
 
-    // 2. per-token scalars, then the tokens in fp32 with the scalars folded in
+    // 2. the basis rows, per-token scalars, then the tokens in fp32 with the scalars folded in
+    {
+        const float4 *src = reinterpret_cast<const float4 *>(U + (size_t)h * r * DK);
+        for (int i = tid; i < r * DK / 4; i += nthr) reinterpret_cast<float4 *>(sut)[i] = src[i];
+    }
     if (KIND != KDA) {
         if (warp == 0) {
             // g_t = a_1 ... a_t by a warp prefix product (n <= 64: two tokens per lane)
@@ -200,7 +205,6 @@ update_window_kernel(ST *__restrict__ S, float *__restrict__ P, const float *__r
     // 5. sketch refresh P[c][m] = sum_i S[i][c] U[i][m] from the stored values: per
     //    basis row m one dot per column and one octet reduction, after which lane
     //    l holds P[c0 + cl][m]; four basis rows per pass bound the rows in flight
-    const float *Uh = U + (size_t)h * r * DK;
     float *Prow = P + ((size_t)head * dv + c0 + cl) * r;
     const bool writer = NC == 8 || (l & 1) == 0;
 #pragma unroll 1
@@ -211,7 +215,7 @@ update_window_kernel(ST *__restrict__ S, float *__restrict__ P, const float *__r
             pm[mm] = 0.f;
             if (m0 + mm < r) {
                 float uv[EPL];
-                lane_channels_global<DK, ST, float>(Uh + (size_t)(m0 + mm) * DK, l, uv);
+                lane_channels_smem<DK, ST>(sut + (m0 + mm) * DK, l, uv);
                 float d[NC];
 #pragma unroll
                 for (int cc = 0; cc < NC; ++cc) d[cc] = dot<EPL>(uv, s[cc]);
@@ -233,7 +237,8 @@ update_window_kernel(ST *__restrict__ S, float *__restrict__ P, const float *__r
 
 static size_t update_smem_bytes(const sketchssm_dims &d, int n) {
     const size_t n4 = (n + 3) & ~3;
-    const size_t fl = (size_t)n * d.dk * (d.kind == SKSSM_KDA ? 2 : 1) + (size_t)n * d.dv + d.dk + 2 * n4;
+    const size_t fl = (size_t)n * d.dk * (d.kind == SKSSM_KDA ? 2 : 1) + (size_t)n * d.dv + d.dk +
+                      (size_t)d.r * d.dk + 2 * n4;
     return fl * sizeof(float);
 }
 

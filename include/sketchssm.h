@@ -151,11 +151,13 @@ int sketchssm_fullread_decode(const sketchssm_dims *dims, void *S, const void *q
 
 /*
  * sketchssm_device_error_count -- kernels never wait without bound: the decode
- * step's wait for its bulk copies gives up after a fixed number of attempts,
- * counts the give-up in a device-side counter and returns without writing its
- * output.  This call synchronises the current device and returns that count
+ * step's and the window update's waits for their bulk copies give up after a
+ * fixed number of attempts, count the give-up in a device-side counter and
+ * return without writing that head's results (the window update also stops
+ * the rest of its CTA's heads, leaving their state and sketch as they were).
+ * This call synchronises the current device and returns the sum of both counts
  * (0 in normal operation; a negative sketchssm_status if a CUDA call fails);
- * reset != 0 clears it.
+ * reset != 0 clears them.
  */
 int sketchssm_device_error_count(int reset);
 

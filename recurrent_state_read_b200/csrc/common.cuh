@@ -212,4 +212,61 @@ __device__ __forceinline__ float octet_sum(float x) {
     return x;
 }
 
+// ---- L2 eviction priority hints ---------------------------------------------
+// The sketch P is re-read by every decode step of a window: it is written and
+// read with an evict-last policy so that it stays in L2 while the state and the
+// buffered tokens stream past.
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ float4 ld_keep(const float *p, uint64_t pol) {
+    float4 a;
+    asm volatile("ld.global.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=f"(a.x), "=f"(a.y), "=f"(a.z), "=f"(a.w)
+                 : "l"(p), "l"(pol));
+    return a;
+}
+__device__ __forceinline__ float ld_keep1(const float *p, uint64_t pol) {
+    float a;
+    asm volatile("ld.global.L2::cache_hint.f32 %0, [%1], %2;" : "=f"(a) : "l"(p), "l"(pol));
+    return a;
+}
+__device__ __forceinline__ void st_keep(float *p, float4 a, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "f"(a.x), "f"(a.y),
+                 "f"(a.z), "f"(a.w), "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ void st_keep1(float *p, float a, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(a), "l"(pol) : "memory");
+}
+
+// Reduce 8 per-lane partials over the whole warp; on return every lane holds all
+// 8 totals.  A reduce-scatter over lane bits 4, 3, 2 (7 shuffles), an all-reduce
+// over bits 1, 0 (2 shuffles), then an all-gather (8 shuffles).
+__device__ __forceinline__ void warp_allreduce8(float (&v)[8], int lane) {
+    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+    float a[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const float send = b4 ? v[m] : v[m + 4];
+        const float keep = b4 ? v[m + 4] : v[m];
+        a[m] = keep + __shfl_xor_sync(FULL, send, 16);
+    }
+    float b[2];
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+        const float send = b3 ? a[m] : a[m + 2];
+        const float keep = b3 ? a[m + 2] : a[m];
+        b[m] = keep + __shfl_xor_sync(FULL, send, 8);
+    }
+    float x = (b2 ? b[1] : b[0]) + __shfl_xor_sync(FULL, b2 ? b[0] : b[1], 4);
+    x += __shfl_xor_sync(FULL, x, 2);
+    x += __shfl_xor_sync(FULL, x, 1);
+    // lane l now holds the total of index (l >> 2) & 7
+#pragma unroll
+    for (int m = 0; m < 8; ++m) v[m] = __shfl_sync(FULL, x, 4 * m);
+}
+
 }  // namespace skssm

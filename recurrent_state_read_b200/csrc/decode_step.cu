@@ -17,20 +17,23 @@
 // A decode step is one memory round trip per head: the head's buffered k and v
 // (and KDA decay) rows are contiguous blocks of the head-major window buffer
 // and arrive by TMA bulk copies into the warp's shared-memory slots, while the
-// query, the per-token scalars (one token per lane), the first eight R rows and
-// the matching sketch rows are loaded into registers at the same time.  The
-// backward pass then runs from shared memory: per token one warp reduction for
-// k . w and one axpy.  Scalar decay is kept as a running scale next to the
-// carried query (w = g w^), so Mamba-2's dot products do not depend on each
-// other.  The wait on the copies is bounded: a give-up is counted in a device
-// flag (sketchssm_device_error_count) and the warp returns.
+// query, the per-token scalars (one token per lane) and the first eight sketch
+// columns are loaded into registers at the same time.  The backward pass then
+// runs from shared memory: per token one warp reduction for k . w and one axpy.
+// Scalar decay is kept as a running scale next to the carried query (w = g w^),
+// so Mamba-2's dot products do not depend on each other and eight of them share
+// one warp all-reduce.  The coefficient rows R (the same for every b) are read
+// after the pass, from L1/L2, so that they hold no registers while the copies
+// are in flight: 64 registers per thread keep eight 4-warp CTAs on an SM.  The
+// wait on the copies is bounded: a give-up is counted in a device flag
+// (sketchssm_device_error_count) and the warp returns.
 #include "internal.h"
 #include "state_tile.cuh"
 
 namespace skssm {
 
-constexpr int DEC_WARPS = 8;  // one head per warp
-constexpr int DEC_RPRE = 8;   // coefficient rows held in registers from the start
+constexpr int DEC_WARPS = 4;  // one head per warp; small CTAs pack the SMs more tightly (measured)
+constexpr int DEC_RPRE = 8;   // sketch columns held in registers from the start; R rows per all-reduce
 constexpr unsigned DEC_WAIT_TRIES = 1u << 22;
 
 __device__ unsigned g_device_error;
@@ -95,25 +98,19 @@ decode_step_kernel(const float *__restrict__ P, const float *__restrict__ R, con
     }
     __syncwarp();
 
-    // registers, all requested before the first wait: query, R rows, sketch rows
-    float w[KPL], rr[DEC_RPRE][KPL], pp[VPL][DEC_RPRE], ob[VPL];
+    // registers, all requested before the first wait: query and the first sketch rows (the
+    // coefficient rows R are shared by the warps of a head index h and come from L1/L2 later)
+    float w[KPL], pp[VPL][DEC_RPRE], ob[VPL];
     load_n<KPL>(qv + (size_t)head * DK + lane * KPL, w);
     const float *Rh = R + (size_t)h * r * DK;
-#pragma unroll
-    for (int m = 0; m < DEC_RPRE; ++m) {
-        if (m < r) load_n<KPL>(Rh + (size_t)m * DK + lane * KPL, rr[m]);
-        else {
-#pragma unroll
-            for (int e = 0; e < KPL; ++e) rr[m][e] = 0.f;
-        }
-    }
     const float *Ph = P + (size_t)head * DV * r;
 #pragma unroll
     for (int e = 0; e < VPL; ++e) {
         const float *row = Ph + (size_t)(lane * VPL + e) * r;
         if ((r & 3) == 0 && r >= DEC_RPRE) {
-            load4(row, pp[e]);
-            load4(row + 4, pp[e] + 4);
+            const float4 a = *reinterpret_cast<const float4 *>(row), b = *reinterpret_cast<const float4 *>(row + 4);
+            pp[e][0] = a.x; pp[e][1] = a.y; pp[e][2] = a.z; pp[e][3] = a.w;
+            pp[e][4] = b.x; pp[e][5] = b.y; pp[e][6] = b.z; pp[e][7] = b.w;
         } else {
 #pragma unroll
             for (int m = 0; m < DEC_RPRE; ++m) pp[e][m] = m < r ? row[m] : 0.f;
@@ -144,6 +141,35 @@ decode_step_kernel(const float *__restrict__ P, const float *__restrict__ R, con
             return;
         }
         phase ^= 1;
+        if constexpr (KIND == MAMBA2) {
+            // w stays q: the dots of eight tokens are independent and share one warp all-reduce
+            for (int t0 = thi; t0 >= tlo; t0 -= 8) {
+                float x[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    x[u] = 0.f;
+                    if (t0 - u >= tlo) {
+                        float kf[KPL];
+                        load_n<KPL>(reinterpret_cast<const QT *>(ks + (t0 - u - tlo) * SL::KB) + lane * KPL, kf);
+#pragma unroll
+                        for (int e = 0; e < KPL; ++e) x[u] = fmaf(kf[e], w[e], x[u]);
+                    }
+                }
+                warp_allreduce8(x, lane);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    if (t0 - u >= tlo) {  // warp-uniform
+                        const int sl = t0 - u - tlo;
+                        float vf[VPL];
+                        load_n<VPL>(reinterpret_cast<const QT *>(vs + sl * SL::VB) + lane * VPL, vf);
+                        const float s = gsc * x[u];  // (k . q) times the decay of the later tokens
+#pragma unroll
+                        for (int e = 0; e < VPL; ++e) ob[e] = fmaf(s, vf[e], ob[e]);
+                        gsc *= __shfl_sync(FULL, a_l, sl);
+                    }
+                }
+            }
+        } else
         for (int t = thi; t >= tlo; --t) {
             const int sl = t - tlo;
             float kf[KPL], vf[VPL];
@@ -180,30 +206,39 @@ decode_step_kernel(const float *__restrict__ P, const float *__restrict__ R, con
         for (int e = 0; e < KPL; ++e) w[e] *= gsc;
     }
 
-    // c = R q~, o = P c + o_buf: the first DEC_RPRE rows from registers, the rest streamed
+    // c = R q~ in blocks of eight rows (one warp all-reduce per block), o = P c + o_buf; the
+    // sketch rows of the first block are already in registers
     float acc[VPL];
 #pragma unroll
     for (int e = 0; e < VPL; ++e) acc[e] = ob[e];
+#pragma unroll 1
+    for (int m0 = 0; m0 < r; m0 += DEC_RPRE) {
+        float c[DEC_RPRE];  // rows m >= r are zero
 #pragma unroll
-    for (int m = 0; m < DEC_RPRE; ++m) {
-        if (m < r) {
-            float p = 0.f;
+        for (int mm = 0; mm < DEC_RPRE; ++mm) {
+            c[mm] = 0.f;
+            if (m0 + mm < r) {
+                float rv[KPL];
+                load_n<KPL>(Rh + (size_t)(m0 + mm) * DK + lane * KPL, rv);
 #pragma unroll
-            for (int e = 0; e < KPL; ++e) p = fmaf(rr[m][e], w[e], p);
-            const float c = warp_sum(p);
-#pragma unroll
-            for (int e = 0; e < VPL; ++e) acc[e] = fmaf(pp[e][m], c, acc[e]);
+                for (int e = 0; e < KPL; ++e) c[mm] = fmaf(rv[e], w[e], c[mm]);
+            }
         }
-    }
-    for (int m = DEC_RPRE; m < r; ++m) {
-        float rv[KPL];
-        load_n<KPL>(Rh + (size_t)m * DK + lane * KPL, rv);
-        float p = 0.f;
+        warp_allreduce8(c, lane);
+        if (m0 == 0) {
 #pragma unroll
-        for (int e = 0; e < KPL; ++e) p = fmaf(rv[e], w[e], p);
-        const float c = warp_sum(p);
+            for (int mm = 0; mm < DEC_RPRE; ++mm)
 #pragma unroll
-        for (int e = 0; e < VPL; ++e) acc[e] = fmaf(Ph[(size_t)(lane * VPL + e) * r + m], c, acc[e]);
+                for (int e = 0; e < VPL; ++e) acc[e] = fmaf(pp[e][mm], c[mm], acc[e]);
+        } else {
+#pragma unroll
+            for (int mm = 0; mm < DEC_RPRE; ++mm)
+                if (m0 + mm < r) {
+#pragma unroll
+                    for (int e = 0; e < VPL; ++e)
+                        acc[e] = fmaf(Ph[(size_t)(lane * VPL + e) * r + m0 + mm], c[mm], acc[e]);
+                }
+        }
     }
     float *oh = o + (size_t)head * DV + lane * VPL;
     if constexpr (VPL == 4) *reinterpret_cast<float4 *>(oh) = make_float4(acc[0], acc[1], acc[2], acc[3]);
@@ -221,7 +256,9 @@ int launch_decode_step(const sketchssm_dims &d, const float *P, const float *R, 
         const int grid = (NH + DEC_WARPS - 1) / DEC_WARPS;
         auto go = [&](auto DVc) -> int {
             constexpr int DV = decltype(DVc)::value;
-            const int jmax = KIND == KDA ? 16 : 32;  // tokens per bulk round trip (<= 32: one per lane)
+            // tokens per bulk round trip (<= 32: one per lane); KDA rows are twice as wide, and fewer
+            // of them per trip keep more warps resident
+            const int jmax = KIND == KDA ? 8 : 32;
             const int jc = j < jmax ? j : jmax;
             const size_t smem = (size_t)DEC_WARPS * DecSlots<KIND, DK, DV, QT>::bytes(jc);
             auto kern = decode_step_kernel<KIND, DK, DV, QT>;
@@ -245,13 +282,15 @@ int launch_decode_step(const sketchssm_dims &d, const float *P, const float *R, 
 
 }  // namespace skssm
 
+int skssm::decode_wait_giveups(bool reset, unsigned *count) {
+    return read_counter(&g_device_error, reset, count);
+}
+
 extern "C" int sketchssm_device_error_count(int reset) {
-    unsigned n = 0;
     if (cudaDeviceSynchronize() != cudaSuccess) return SKSSM_ERR_CUDA;
-    if (cudaMemcpyFromSymbol(&n, skssm::g_device_error, sizeof(n)) != cudaSuccess) return SKSSM_ERR_CUDA;
-    if (reset && n) {
-        const unsigned zero = 0;
-        if (cudaMemcpyToSymbol(skssm::g_device_error, &zero, sizeof(zero)) != cudaSuccess) return SKSSM_ERR_CUDA;
-    }
-    return (int)n;
+    unsigned dec = 0, upd = 0;
+    if (skssm::decode_wait_giveups(reset != 0, &dec) != SKSSM_OK ||
+        skssm::update_wait_giveups(reset != 0, &upd) != SKSSM_OK)
+        return SKSSM_ERR_CUDA;
+    return (int)(dec + upd);
 }

@@ -45,6 +45,21 @@ inline int launch_status() {
 int launch_update_window(const sketchssm_dims &d, void *S, float *P, const float *U, const void *k,
                          const void *v, const float *alpha, const float *beta, int n_tokens,
                          cudaStream_t stream);
+// Counts of bounded in-kernel waits that gave up (window update, decode step); reset clears them.
+int update_wait_giveups(bool reset, unsigned *count);
+int decode_wait_giveups(bool reset, unsigned *count);
+
+// Read (and optionally clear) a __device__ counter from the host.
+template <typename T>
+inline int read_counter(const T *symbol, bool reset, unsigned *count) {
+    *count = 0;
+    if (cudaMemcpyFromSymbol(count, *symbol, sizeof(unsigned)) != cudaSuccess) return SKSSM_ERR_CUDA;
+    if (reset && *count) {
+        const unsigned zero = 0;
+        if (cudaMemcpyToSymbol(*symbol, &zero, sizeof(zero)) != cudaSuccess) return SKSSM_ERR_CUDA;
+    }
+    return SKSSM_OK;
+}
 int launch_fullread(const sketchssm_dims &d, void *S, const void *q, const void *k, const void *v,
                     const float *alpha, const float *beta, float *o, cudaStream_t stream);
 int launch_decode_step(const sketchssm_dims &d, const float *P, const float *R, const void *q,

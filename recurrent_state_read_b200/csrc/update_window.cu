@@ -28,6 +28,9 @@
 namespace skssm {
 
 constexpr int UPD_NC = 8;  // value columns per lane (state_tile.cuh)
+constexpr int PER_NC = 4;      // the same for the persistent kernel
+constexpr int PER_STAGES = 1;  // shared-memory stages per persistent CTA: with one stage more CTAs fit on an
+                               // SM, which hides the copies better than a deeper pipeline per CTA (measured)
 
 // Inclusive prefix product across the warp.
 __device__ __forceinline__ float warp_prefix_product(float x, int lane) {
@@ -75,6 +78,99 @@ __device__ __forceinline__ void stage_rows(const T *__restrict__ src, size_t row
     }
 }
 
+// Steps shared by both window-update kernels, for one head whose state is in
+// registers: apply the n staged tokens in order, scale, round to the storage
+// type, store the state once, and refresh the sketch from the same registers.
+template <int KIND, int DK, typename ST, int NC>
+__device__ __forceinline__ void apply_store_refresh(float (&s)[NC][DK / 8], const float *sk, const float *su,
+                                                    const float *sv, const float *sg, const float *sut,
+                                                    const float *ss2, ST *__restrict__ S, float *__restrict__ P,
+                                                    int head, int dv, int r, int n, int c0, int l, int lane) {
+    using TL = TileLayout<DK, ST>;
+    constexpr int EPL = TL::EPL;
+    const int cl = NC == 8 ? l : l >> 1;  // the column whose reduced values this lane holds
+    // the buffered tokens, in order
+    for (int t = 0; t < n; ++t) {
+        float kv[EPL];
+        lane_channels_smem<DK, ST>(sk + t * DK, l, kv);
+        if (KIND == MAMBA2) {
+            float vv[NC];
+#pragma unroll
+            for (int c4 = 0; c4 < NC; c4 += 4) {
+                const float4 a = *reinterpret_cast<const float4 *>(sv + t * dv + c0 + c4);
+                vv[c4] = a.x; vv[c4 + 1] = a.y; vv[c4 + 2] = a.z; vv[c4 + 3] = a.w;
+            }
+#pragma unroll
+            for (int cc = 0; cc < NC; ++cc) axpy<EPL>(s[cc], kv, vv[cc]);
+        } else {
+            float d[NC];
+#pragma unroll
+            for (int cc = 0; cc < NC; ++cc) d[cc] = dot<EPL>(kv, s[cc]);
+            float dsum;
+            if constexpr (NC == 8) dsum = octet_reduce_scatter(d, lane);
+            else dsum = octet_reduce4(d, lane);
+            const float vc = sv[t * dv + c0 + cl];
+            const float u = KIND == GDN ? vc - ss2[t] * dsum : vc - dsum;
+            float uu[NC];
+            if constexpr (NC == 8) octet_all_gather(u, uu);
+            else octet_all_gather4(u, uu);
+            if (KIND == KDA) lane_channels_smem<DK, ST>(su + t * DK, l, kv);
+#pragma unroll
+            for (int cc = 0; cc < NC; ++cc) axpy<EPL>(s[cc], kv, uu[cc]);
+        }
+    }
+
+    // final scale, storage rounding, one store of the state
+    if (KIND != KDA) {
+        const float gam = sg[0];
+#pragma unroll
+        for (int cc = 0; cc < NC; ++cc)
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) s[cc][e] = as_stored<ST>(s[cc][e] * gam);
+    } else {
+        float gv[EPL];
+        lane_channels_smem<DK, ST>(sg, l, gv);
+#pragma unroll
+        for (int cc = 0; cc < NC; ++cc)
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) s[cc][e] = as_stored<ST>(s[cc][e] * gv[e]);
+    }
+    if (n > 0) store_tile<DK, ST, NC>(S + (size_t)head * dv * DK, c0, l, s);
+
+    // sketch refresh P[c][m] = sum_i S[i][c] U[i][m] from the stored values: per
+    //    basis row m one dot per column and one octet reduction, after which lane
+    //    l holds P[c0 + cl][m]; four basis rows per pass bound the rows in flight
+    float *Prow = P + ((size_t)head * dv + c0 + cl) * r;
+    const uint64_t keep = l2_evict_last_policy();  // the decode steps re-read P from L2
+    const bool writer = NC == 8 || (l & 1) == 0;
+#pragma unroll 1
+    for (int m0 = 0; m0 < r; m0 += 4) {
+        float pm[4];
+#pragma unroll
+        for (int mm = 0; mm < 4; ++mm) {
+            pm[mm] = 0.f;
+            if (m0 + mm < r) {
+                float uv[EPL];
+                lane_channels_smem<DK, ST>(sut + (m0 + mm) * DK, l, uv);
+                float d[NC];
+#pragma unroll
+                for (int cc = 0; cc < NC; ++cc) d[cc] = dot<EPL>(uv, s[cc]);
+                if constexpr (NC == 8) pm[mm] = octet_reduce_scatter(d, lane);
+                else pm[mm] = octet_reduce4(d, lane);
+            }
+        }
+        if (writer) {
+            if ((r & 3) == 0) {
+                st_keep(Prow + m0, make_float4(pm[0], pm[1], pm[2], pm[3]), keep);
+            } else {
+#pragma unroll
+                for (int mm = 0; mm < 4; ++mm)
+                    if (m0 + mm < r) st_keep1(Prow + m0 + mm, pm[mm], keep);
+            }
+        }
+    }
+}
+
 template <int KIND, int DK, typename ST, typename QT, int NC>
 __global__ void __launch_bounds__(256)
 update_window_kernel(ST *__restrict__ S, float *__restrict__ P, const float *__restrict__ U,
@@ -91,7 +187,6 @@ update_window_kernel(ST *__restrict__ S, float *__restrict__ P, const float *__r
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int l = lane & 7, g = lane >> 3;
     const int c0 = warp * 4 * NC + g * NC;
-    const int cl = NC == 8 ? l : l >> 1;  // the column whose reduced values this lane holds
     const int nthr = blockDim.x;
 
     // shared memory, each array a multiple of 4 floats: dot vectors, update
@@ -154,84 +249,242 @@ update_window_kernel(ST *__restrict__ S, float *__restrict__ P, const float *__r
     }
     __syncthreads();
 
-    // 3. the buffered tokens, in order
-    for (int t = 0; t < n; ++t) {
-        float kv[EPL];
-        lane_channels_smem<DK, ST>(sk + t * DK, l, kv);
-        if (KIND == MAMBA2) {
-            float vv[NC];
-#pragma unroll
-            for (int c4 = 0; c4 < NC; c4 += 4) {
-                const float4 a = *reinterpret_cast<const float4 *>(sv + t * dv + c0 + c4);
-                vv[c4] = a.x; vv[c4 + 1] = a.y; vv[c4 + 2] = a.z; vv[c4 + 3] = a.w;
+    apply_store_refresh<KIND, DK, ST, NC>(s, sk, su, sv, sg, sut, ss2, S, P, head, dv, r, n, c0, l, lane);
+}
+
+// ---------------------------------------------------------------------------
+// Persistent, pipelined variant.  A CTA owns a contiguous run of heads in
+// (h, b) order.  Each head's state (one contiguous dv x dk block) and its window
+// tokens (contiguous blocks of the head-major buffer) arrive by TMA bulk copies
+// into one of NS shared-memory stages, signalled by that stage's mbarrier; while
+// the CTA applies head i's tokens from registers, heads i+1 .. i+NS-1 are in
+// flight.  A stage is refilled as soon as the CTA has moved its head into
+// registers and fp32 staging.  Waits are bounded: a give-up is counted
+// (sketchssm_device_error_count) and the CTA returns.
+// ---------------------------------------------------------------------------
+
+__device__ unsigned g_update_wait_giveups;
+constexpr unsigned UPD_WAIT_TRIES = 1u << 22;
+
+__device__ __forceinline__ unsigned upd_smem(const void *p) { return (unsigned)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ bool upd_wait(const uint64_t *bar, int parity) {
+    for (unsigned it = 0; it < UPD_WAIT_TRIES; ++it) {
+        unsigned done;
+        asm volatile(
+            "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }\n"
+            : "=r"(done)
+            : "r"(upd_smem(bar)), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+
+__device__ __forceinline__ void upd_bulk(void *dst, const void *src, int bytes, const uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                     upd_smem(dst)),
+                 "l"(src), "r"(bytes), "r"(upd_smem(bar))
+                 : "memory");
+}
+
+__host__ __device__ inline int up16(int x) { return (x + 15) & ~15; }
+
+// Byte offsets of the persistent kernel's shared memory (host and device agree).
+struct PerLayout {
+    int stage_bytes, st, kr, vr, ar;  // inside a stage: state, raw k, raw v, raw decay (KDA)
+    int stages;                       // first stage (NS stages follow, stage_bytes apart)
+    int sk, su, sv, sg, sut, ss2, total;
+};
+
+__host__ __device__ inline PerLayout per_layout(int kind, int DK, int dv, int r, int n, int sbytes, int qbytes,
+                                                int ns) {
+    PerLayout L;
+    int t = 0;
+    L.st = t; t += up16(dv * DK * sbytes);
+    L.kr = t; t += up16(n * DK * qbytes);
+    L.vr = t; t += up16(n * dv * qbytes);
+    L.ar = t; t += kind == KDA ? up16(n * DK * 4) : 0;
+    L.stage_bytes = t;
+    int off = 16 * 2;  // two mbarriers, 16 bytes apart
+    L.stages = off; off += ns * t;
+    L.sk = off; off += up16(n * DK * 4);
+    L.su = off; off += kind == KDA ? up16(n * DK * 4) : 0;
+    L.sv = off; off += up16(n * dv * 4);
+    L.sg = off; off += up16(DK * 4);
+    L.sut = off; off += up16(r * DK * 4);
+    L.ss2 = off; off += up16(n * 4);
+    L.total = off;
+    return L;
+}
+
+template <int KIND, int DK, typename ST, typename QT, int NC>
+__global__ void __launch_bounds__(256)
+update_window_persistent(ST *__restrict__ S, float *__restrict__ P, const float *__restrict__ U,
+                         const QT *__restrict__ kbuf, const QT *__restrict__ vbuf,
+                         const float *__restrict__ abuf, const float *__restrict__ bbuf, int B, int H, int dv,
+                         int r, int n, int W, int ns) {
+    using TL = TileLayout<DK, ST>;
+    constexpr int EPL = TL::EPL;
+    extern __shared__ __align__(128) float psm_f[];
+    char *smem = reinterpret_cast<char *>(psm_f);
+    const PerLayout L = per_layout(KIND, DK, dv, r, n, sizeof(ST), sizeof(QT), ns);
+    const int NH = B * H;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int l = lane & 7, g = lane >> 3;
+    const int c0 = warp * 4 * NC + g * NC;
+    const int nthr = blockDim.x;
+
+    const int per = (NH + gridDim.x - 1) / gridDim.x;
+    const int w_begin = blockIdx.x * per;
+    const int w_end = min(NH, w_begin + per);
+    auto head_of = [&](int w) { return (w % B) * H + w / B; };
+
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
+    float *sk = reinterpret_cast<float *>(smem + L.sk);
+    float *su = reinterpret_cast<float *>(smem + L.su);
+    float *sv = reinterpret_cast<float *>(smem + L.sv);
+    float *sg = reinterpret_cast<float *>(smem + L.sg);
+    float *sut = reinterpret_cast<float *>(smem + L.sut);
+    float *ss2 = reinterpret_cast<float *>(smem + L.ss2);
+    const int state_bytes = dv * DK * (int)sizeof(ST);
+    const int kbytes = n * DK * (int)sizeof(QT), vbytes = n * dv * (int)sizeof(QT);
+    const int abytes = KIND == KDA ? n * DK * 4 : 0;
+
+    auto issue = [&](int w, int stage) {  // one thread
+        char *sb = smem + L.stages + stage * L.stage_bytes;
+        const int head = head_of(w);
+        uint64_t *bar = bars + 2 * stage;
+        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(upd_smem(bar)),
+                     "r"(state_bytes + kbytes + vbytes + abytes)
+                     : "memory");
+        upd_bulk(sb + L.st, S + (size_t)head * dv * DK, state_bytes, bar);
+        if (n > 0) {
+            upd_bulk(sb + L.kr, kbuf + (size_t)head * W * DK, kbytes, bar);
+            upd_bulk(sb + L.vr, vbuf + (size_t)head * W * dv, vbytes, bar);
+            if (KIND == KDA) upd_bulk(sb + L.ar, abuf + (size_t)head * W * DK, abytes, bar);
+        }
+    };
+
+    if (tid == 0) {
+        for (int st = 0; st < ns; ++st)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(upd_smem(bars + 2 * st)) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    __syncthreads();
+    if (tid == 0)
+        for (int st = 0; st < ns && w_begin + st < w_end; ++st) issue(w_begin + st, st);
+
+    // per-token scalars of the current head: lanes t and t + 32 of every warp
+    auto load_scalars = [&](int w, float &a0, float &a1, float &b0, float &b1) {
+        const size_t base = (size_t)head_of(w) * W;
+        a0 = a1 = b0 = b1 = 1.f;
+        if (KIND != KDA) {
+            if (lane < n) a0 = abuf[base + lane];
+            if (lane + 32 < n) a1 = abuf[base + lane + 32];
+        }
+        if (KIND != MAMBA2) {
+            if (lane < n) b0 = bbuf[base + lane];
+            if (lane + 32 < n) b1 = bbuf[base + lane + 32];
+        }
+    };
+    float a0, a1, b0, b1;
+    if (w_begin < w_end) load_scalars(w_begin, a0, a1, b0, b1);
+
+    int h_prev = -1;
+    for (int w = w_begin, it = 0; w < w_end; ++w, ++it) {
+        const int stage = it % ns;
+        const int parity = (it / ns) & 1;
+        const int head = head_of(w), h = w / B;
+        const char *sb = smem + L.stages + stage * L.stage_bytes;
+        const bool landed = upd_wait(bars + 2 * stage, parity);
+        // one decision for the whole CTA; the barrier also orders the previous
+        // head's reads of the fp32 staging before this head's writes
+        if (__syncthreads_or(!landed)) {
+            if (tid == 0) {  // count the give-up, then drain the copies still in flight (bounded)
+                atomicAdd(&g_update_wait_giveups, 1u);
+                for (int k2 = 0; k2 < ns && w + k2 < w_end; ++k2)
+                    upd_wait(bars + 2 * ((it + k2) % ns), ((it + k2) / ns) & 1);
             }
+            __syncthreads();
+            return;
+        }
+
+        // state to registers
+        float s[NC][EPL];
+        const ST *st = reinterpret_cast<const ST *>(sb + L.st);
 #pragma unroll
-            for (int cc = 0; cc < NC; ++cc) axpy<EPL>(s[cc], kv, vv[cc]);
+        for (int cc = 0; cc < NC; ++cc)
+#pragma unroll
+            for (int q = 0; q < TL::NQ; ++q)
+                load16<ST>(st + (size_t)(c0 + cc) * DK + TL::chan(l, q, 0), &s[cc][q * TL::VEC]);
+        if (h != h_prev) {
+            const float4 *src = reinterpret_cast<const float4 *>(U + (size_t)h * r * DK);
+            for (int i = tid; i < r * DK / 4; i += nthr) reinterpret_cast<float4 *>(sut)[i] = src[i];
+            h_prev = h;
+        }
+        const QT *kr = reinterpret_cast<const QT *>(sb + L.kr);
+        const QT *vr = reinterpret_cast<const QT *>(sb + L.vr);
+        if (KIND != KDA) {
+            // every warp forms g_t = a_1 ... a_t itself (prefix product over lanes t, t + 32)
+            const float p0 = warp_prefix_product(a0, lane);
+            const float p1 = warp_prefix_product(a1, lane) * __shfl_sync(FULL, p0, 31);
+            const float s_lo = b0 / p0, s_hi = b1 / p1;  // b_t / g_t
+            if (warp == 0) {
+                const float g_lo = __shfl_sync(FULL, p0, (n >= 1 && n <= 32) ? n - 1 : 31);
+                const float g_hi = __shfl_sync(FULL, p1, n > 32 ? n - 33 : 0);
+                if (lane == 0) sg[0] = n == 0 ? 1.f : (n <= 32 ? g_lo : g_hi);
+                if (KIND == GDN) {
+                    if (lane < n) ss2[lane] = b0;
+                    if (lane + 32 < n) ss2[lane + 32] = b1;
+                }
+            }
+            for (int idx = tid * 4; idx < n * DK; idx += nthr * 4) {
+                float f[4];
+                load4(kr + idx, f);
+                *reinterpret_cast<float4 *>(sk + idx) = make_float4(f[0], f[1], f[2], f[3]);
+            }
+            const int vtot = n * dv;  // warp-uniform trips: every lane takes part in the shuffles
+            for (int base = warp * 128; base < vtot; base += (nthr / 32) * 128) {
+                const int idx = base + lane * 4;
+                const int t = (idx < vtot ? idx : vtot - 4) / dv;
+                const float slo = __shfl_sync(FULL, s_lo, t & 31), shi = __shfl_sync(FULL, s_hi, t & 31);
+                if (idx < vtot) {
+                    const float sc = t < 32 ? slo : shi;
+                    float f[4];
+                    load4(vr + idx, f);
+                    *reinterpret_cast<float4 *>(sv + idx) = make_float4(f[0] * sc, f[1] * sc, f[2] * sc, f[3] * sc);
+                }
+            }
         } else {
-            float d[NC];
-#pragma unroll
-            for (int cc = 0; cc < NC; ++cc) d[cc] = dot<EPL>(kv, s[cc]);
-            float dsum;
-            if constexpr (NC == 8) dsum = octet_reduce_scatter(d, lane);
-            else dsum = octet_reduce4(d, lane);
-            const float vc = sv[t * dv + c0 + cl];
-            const float u = KIND == GDN ? vc - ss2[t] * dsum : vc - dsum;
-            float uu[NC];
-            if constexpr (NC == 8) octet_all_gather(u, uu);
-            else octet_all_gather4(u, uu);
-            if (KIND == KDA) lane_channels_smem<DK, ST>(su + t * DK, l, kv);
-#pragma unroll
-            for (int cc = 0; cc < NC; ++cc) axpy<EPL>(s[cc], kv, uu[cc]);
-        }
-    }
-
-    // 4. final scale, storage rounding, one store of the state
-    if (KIND != KDA) {
-        const float gam = sg[0];
-#pragma unroll
-        for (int cc = 0; cc < NC; ++cc)
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) s[cc][e] = as_stored<ST>(s[cc][e] * gam);
-    } else {
-        float gv[EPL];
-        lane_channels_smem<DK, ST>(sg, l, gv);
-#pragma unroll
-        for (int cc = 0; cc < NC; ++cc)
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) s[cc][e] = as_stored<ST>(s[cc][e] * gv[e]);
-    }
-    if (n > 0) store_tile<DK, ST, NC>(S + (size_t)head * dv * DK, c0, l, s);
-
-    // 5. sketch refresh P[c][m] = sum_i S[i][c] U[i][m] from the stored values: per
-    //    basis row m one dot per column and one octet reduction, after which lane
-    //    l holds P[c0 + cl][m]; four basis rows per pass bound the rows in flight
-    float *Prow = P + ((size_t)head * dv + c0 + cl) * r;
-    const bool writer = NC == 8 || (l & 1) == 0;
-#pragma unroll 1
-    for (int m0 = 0; m0 < r; m0 += 4) {
-        float pm[4];
-#pragma unroll
-        for (int mm = 0; mm < 4; ++mm) {
-            pm[mm] = 0.f;
-            if (m0 + mm < r) {
-                float uv[EPL];
-                lane_channels_smem<DK, ST>(sut + (m0 + mm) * DK, l, uv);
-                float d[NC];
-#pragma unroll
-                for (int cc = 0; cc < NC; ++cc) d[cc] = dot<EPL>(uv, s[cc]);
-                if constexpr (NC == 8) pm[mm] = octet_reduce_scatter(d, lane);
-                else pm[mm] = octet_reduce4(d, lane);
+            const float *ar = reinterpret_cast<const float *>(sb + L.ar);
+            if (warp == 0) {
+                if (lane < n) ss2[lane] = b0;
+                if (lane + 32 < n) ss2[lane + 32] = b1;
+            }
+            for (int i = tid; i < DK; i += nthr) {
+                float gam = 1.f;
+                for (int t = 0; t < n; ++t) {
+                    gam *= ar[t * DK + i];
+                    const float bt = __shfl_sync(__activemask(), t < 32 ? b0 : b1, t & 31);
+                    const float k = ld1(kr + t * DK + i);
+                    sk[t * DK + i] = k * gam;
+                    su[t * DK + i] = bt * k * (1.f / gam);
+                }
+                sg[i] = gam;
+            }
+            for (int idx = tid * 4; idx < n * dv; idx += nthr * 4) {
+                float f[4];
+                load4(vr + idx, f);
+                *reinterpret_cast<float4 *>(sv + idx) = make_float4(f[0], f[1], f[2], f[3]);
             }
         }
-        if (writer) {
-            if ((r & 3) == 0) {
-                *reinterpret_cast<float4 *>(Prow + m0) = make_float4(pm[0], pm[1], pm[2], pm[3]);
-            } else {
-#pragma unroll
-                for (int mm = 0; mm < 4; ++mm)
-                    if (m0 + mm < r) Prow[m0 + mm] = pm[mm];
-            }
-        }
+        if (w + 1 < w_end) load_scalars(w + 1, a0, a1, b0, b1);  // in flight behind this head
+        __syncthreads();  // the stage is consumed; the fp32 staging is ready
+        if (tid == 0 && w + ns < w_end) issue(w + ns, stage);
+
+        apply_store_refresh<KIND, DK, ST, NC>(s, sk, su, sv, sg, sut, ss2, S, P, head, dv, r, n, c0, l, lane);
     }
 }
 
@@ -245,28 +498,54 @@ static size_t update_smem_bytes(const sketchssm_dims &d, int n) {
 int launch_update_window(const sketchssm_dims &d, void *S, float *P, const float *U, const void *k,
                          const void *v, const float *alpha, const float *beta, int n,
                          cudaStream_t stream) {
-    const size_t smem = update_smem_bytes(d, n);
-    if (smem > 227 * 1024) return SKSSM_ERR_DIMS;
+    constexpr int LIMIT = 227 * 1024;
     return dispatch(d, [&](auto K, auto D, auto *sp, auto *qp) -> int {
         using ST = std::remove_pointer_t<decltype(sp)>;
         using QT = std::remove_pointer_t<decltype(qp)>;
         constexpr int KIND = decltype(K)::value, DK = decltype(D)::value;
+        const int NH = d.B * d.H;
+        // persistent kernel, state and tokens by bulk copies; one CTA per head if its layout does not fit
+        const int ns = PER_STAGES;
+        const PerLayout L = per_layout(KIND, DK, d.dv, d.r, n, sizeof(ST), sizeof(QT), ns);
+        if (L.total <= LIMIT) {
+            auto kern = update_window_persistent<KIND, DK, ST, QT, PER_NC>;
+            const int threads = d.dv * 8 / PER_NC;
+            static bool opted_in = false;
+            if (!opted_in) {
+                if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LIMIT) != cudaSuccess)
+                    return SKSSM_ERR_CUDA;
+                opted_in = true;
+            }
+            int dev = 0, sms = 0, per_sm = 0;
+            if (cudaGetDevice(&dev) != cudaSuccess ||
+                cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, L.total) != cudaSuccess)
+                return SKSSM_ERR_CUDA;
+            if (per_sm >= 1) {
+                const int grid = NH < sms * per_sm ? NH : sms * per_sm;
+                kern<<<grid, threads, L.total, stream>>>(static_cast<ST *>(S), P, U, static_cast<const QT *>(k),
+                                                         static_cast<const QT *>(v), alpha, beta, d.B, d.H, d.dv,
+                                                         d.r, n, d.W, ns);
+                return launch_status();
+            }
+        }
+        // one CTA per head
+        const int threads = d.dv * 8 / UPD_NC;
+        const size_t smem = update_smem_bytes(d, n);
+        if (smem > (size_t)LIMIT) return SKSSM_ERR_DIMS;
         auto kern = update_window_kernel<KIND, DK, ST, QT, UPD_NC>;
-        // Opt in to the largest dynamic shared memory once per instantiation, so
-        // that later calls (for example inside a graph capture) make no attribute call.
         static bool opted_in = false;
         if (!opted_in) {
-            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-                cudaSuccess)
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LIMIT) != cudaSuccess)
                 return SKSSM_ERR_CUDA;
             opted_in = true;
         }
-        const int NH = d.B * d.H;
-        kern<<<NH, d.dv * 8 / UPD_NC, smem, stream>>>(static_cast<ST *>(S), P, U, static_cast<const QT *>(k),
-                                                      static_cast<const QT *>(v), alpha, beta, d.B, d.H, d.dv,
-                                                      d.r, n, d.W);
+        kern<<<NH, threads, smem, stream>>>(static_cast<ST *>(S), P, U, static_cast<const QT *>(k),
+                                            static_cast<const QT *>(v), alpha, beta, d.B, d.H, d.dv, d.r, n, d.W);
         return launch_status();
     });
 }
+
+int update_wait_giveups(bool reset, unsigned *count) { return read_counter(&g_update_wait_giveups, reset, count); }
 
 }  // namespace skssm

@@ -57,6 +57,7 @@ CASES = [
     ("gdn", 128, 128, 8, 16, torch.bfloat16, torch.bfloat16),
     ("kda", 128, 128, 8, 16, torch.bfloat16, torch.bfloat16),
     ("gdn", 64, 64, 4, 8, torch.bfloat16, torch.float32),
+    ("kda", 128, 128, 128, 64, torch.float32, torch.float32),  # largest layout: one CTA per head
 ]
 
 
@@ -143,6 +144,32 @@ def test_fullread_decode(case):
     bf = sdt == torch.bfloat16
     assert state_err(to_logical(S), Sref) <= (BF16_STATE_TOL if bf else STATE_TOL)
     assert rel_l2(outs.reshape(T, B * H, dv).cpu(), Oref) <= (BF16_OUT_TOL if bf else TIGHT_OUT)
+
+
+@pytest.mark.parametrize("kind", ["mamba2", "gdn", "kda"])
+def test_update_window_many_heads_per_cta(kind):
+    """2100 heads (B=7, H=300): the persistent window update runs several heads per CTA, across
+    changes of h (new basis rows) inside one CTA; every head is checked."""
+    import recurrent_state_read_b200 as rs
+
+    dk = dv = 64
+    r, W = 8, 8
+    cfg, d, S0, U, R, tok = _setup(kind, dk, dv, r, W, torch.float32, torch.float32, B=7, H=300, seed=3)
+    B, H = d.B, d.H
+    Uh = oracle.per_head(U, H, np.arange(B * H))
+    ft = flat_tokens(tok)
+    dev = to_window(to_device(tok))
+    for n in (0, 5, W):
+        S = to_gpu_state(S0, B, H)
+        P = torch.full((B, H, dv, r), float("nan"), device="cuda")
+        rs.sketchssm_update_window(d, S, P, U.transpose(1, 2).contiguous().cuda(), dev["k"], dev["v"],
+                                   dev["alpha"], dev["beta"], n)
+        torch.cuda.synchronize()
+        sl = slice(0, n)
+        Sref, Pref = oracle.update_window(kind, S0, Uh, ft["k"][sl] if n else None, ft["v"][sl],
+                                          ft["alpha"][sl], None if ft["beta"] is None else ft["beta"][sl])
+        assert state_err(to_logical(S), Sref) <= STATE_TOL, n
+        assert state_err(P.reshape(B * H, dv, r).double().cpu().numpy(), Pref) <= STATE_TOL, n
 
 
 def test_complete_basis_sketch_is_exact_read():

@@ -35,6 +35,7 @@ namespace skssm {
 constexpr int DEC_WARPS = 4;  // one head per warp; small CTAs pack the SMs more tightly (measured)
 constexpr int DEC_RPRE = 8;   // sketch columns held in registers from the start; R rows per all-reduce
 constexpr unsigned DEC_WAIT_TRIES = 1u << 22;
+constexpr int DEC_PERSIST_MIN_WARPS = 12;  // fewest resident warps per SM for the pipelined kernel (measured crossover)
 
 __device__ unsigned g_device_error;
 
@@ -72,6 +73,76 @@ template <int N, typename T>
 __device__ __forceinline__ void load_n(const T *p, float *out) {
     if constexpr (N == 4) load4(p, out);
     else load2(p, out);
+}
+
+// The backward pass over one chunk of buffered tokens held in shared memory
+// (slots 0 .. nt-1, oldest first; ks/vs/as their k, v and KDA decay rows), newest
+// first: per token x = k . w, o_buf += b x v, w <- M^T w.  Lane t holds the chunk's
+// token-t scalars a_l, b_l.  For scalar decay w is kept as gsc * w^.
+template <int KIND, int DK, int DV, typename QT>
+__device__ __forceinline__ void backward_chunk(const char *ks, const char *vs, const char *as, int nt, float a_l,
+                                               float b_l, float (&w)[DK / 32], float (&ob)[DV / 32], float &gsc,
+                                               int lane) {
+    using SL = DecSlots<KIND, DK, DV, QT>;
+    constexpr int KPL = DK / 32, VPL = DV / 32;
+    if constexpr (KIND == MAMBA2) {
+        // w stays q: the dots of eight tokens are independent and share one warp all-reduce
+        for (int t0 = nt - 1; t0 >= 0; t0 -= 8) {
+            float x[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                x[u] = 0.f;
+                if (t0 - u >= 0) {
+                    float kf[KPL];
+                    load_n<KPL>(reinterpret_cast<const QT *>(ks + (t0 - u) * SL::KB) + lane * KPL, kf);
+#pragma unroll
+                    for (int e = 0; e < KPL; ++e) x[u] = fmaf(kf[e], w[e], x[u]);
+                }
+            }
+            warp_allreduce8(x, lane);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (t0 - u >= 0) {  // warp-uniform
+                    const int sl = t0 - u;
+                    float vf[VPL];
+                    load_n<VPL>(reinterpret_cast<const QT *>(vs + sl * SL::VB) + lane * VPL, vf);
+                    const float s = gsc * x[u];  // (k . q) times the decay of the later tokens
+#pragma unroll
+                    for (int e = 0; e < VPL; ++e) ob[e] = fmaf(s, vf[e], ob[e]);
+                    gsc *= __shfl_sync(FULL, a_l, sl);
+                }
+            }
+        }
+    } else {
+        for (int sl = nt - 1; sl >= 0; --sl) {
+            float kf[KPL], vf[VPL];
+            load_n<KPL>(reinterpret_cast<const QT *>(ks + sl * SL::KB) + lane * KPL, kf);
+            load_n<VPL>(reinterpret_cast<const QT *>(vs + sl * SL::VB) + lane * VPL, vf);
+            const float at = __shfl_sync(FULL, a_l, sl), bt = __shfl_sync(FULL, b_l, sl);
+            float x = 0.f;
+#pragma unroll
+            for (int e = 0; e < KPL; ++e) x = fmaf(kf[e], w[e], x);
+            x = warp_sum(x);  // k . w (k . w^ for scalar decay)
+            if (KIND == KDA) {
+                const float s = bt * x;
+#pragma unroll
+                for (int e = 0; e < VPL; ++e) ob[e] = fmaf(s, vf[e], ob[e]);
+                float a[KPL];
+                load_n<KPL>(reinterpret_cast<const float *>(as + sl * SL::AB) + lane * KPL, a);
+#pragma unroll
+                for (int e = 0; e < KPL; ++e) w[e] = a[e] * fmaf(-s, kf[e], w[e]);
+            } else {
+                const float s = bt * gsc * x;  // b (k . w), w = gsc w^
+#pragma unroll
+                for (int e = 0; e < VPL; ++e) ob[e] = fmaf(s, vf[e], ob[e]);
+                if (KIND == GDN) {
+#pragma unroll
+                    for (int e = 0; e < KPL; ++e) w[e] = fmaf(-bt * x, kf[e], w[e]);  // w^ -= b (k . w^) k
+                }
+                gsc *= at;
+            }
+        }
+    }
 }
 
 template <int KIND, int DK, int DV, typename QT>
@@ -141,64 +212,7 @@ decode_step_kernel(const float *__restrict__ P, const float *__restrict__ R, con
             return;
         }
         phase ^= 1;
-        if constexpr (KIND == MAMBA2) {
-            // w stays q: the dots of eight tokens are independent and share one warp all-reduce
-            for (int t0 = thi; t0 >= tlo; t0 -= 8) {
-                float x[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    x[u] = 0.f;
-                    if (t0 - u >= tlo) {
-                        float kf[KPL];
-                        load_n<KPL>(reinterpret_cast<const QT *>(ks + (t0 - u - tlo) * SL::KB) + lane * KPL, kf);
-#pragma unroll
-                        for (int e = 0; e < KPL; ++e) x[u] = fmaf(kf[e], w[e], x[u]);
-                    }
-                }
-                warp_allreduce8(x, lane);
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    if (t0 - u >= tlo) {  // warp-uniform
-                        const int sl = t0 - u - tlo;
-                        float vf[VPL];
-                        load_n<VPL>(reinterpret_cast<const QT *>(vs + sl * SL::VB) + lane * VPL, vf);
-                        const float s = gsc * x[u];  // (k . q) times the decay of the later tokens
-#pragma unroll
-                        for (int e = 0; e < VPL; ++e) ob[e] = fmaf(s, vf[e], ob[e]);
-                        gsc *= __shfl_sync(FULL, a_l, sl);
-                    }
-                }
-            }
-        } else
-        for (int t = thi; t >= tlo; --t) {
-            const int sl = t - tlo;
-            float kf[KPL], vf[VPL];
-            load_n<KPL>(reinterpret_cast<const QT *>(ks + sl * SL::KB) + lane * KPL, kf);
-            load_n<VPL>(reinterpret_cast<const QT *>(vs + sl * SL::VB) + lane * VPL, vf);
-            const float at = __shfl_sync(FULL, a_l, sl), bt = __shfl_sync(FULL, b_l, sl);
-            float x = 0.f;
-#pragma unroll
-            for (int e = 0; e < KPL; ++e) x = fmaf(kf[e], w[e], x);
-            x = warp_sum(x);  // k . w (k . w^ for scalar decay)
-            if (KIND == KDA) {
-                const float s = bt * x;
-#pragma unroll
-                for (int e = 0; e < VPL; ++e) ob[e] = fmaf(s, vf[e], ob[e]);
-                float a[KPL];
-                load_n<KPL>(reinterpret_cast<const float *>(as + sl * SL::AB) + lane * KPL, a);
-#pragma unroll
-                for (int e = 0; e < KPL; ++e) w[e] = a[e] * fmaf(-s, kf[e], w[e]);
-            } else {
-                const float s = bt * gsc * x;  // b (k . w), w = gsc w^
-#pragma unroll
-                for (int e = 0; e < VPL; ++e) ob[e] = fmaf(s, vf[e], ob[e]);
-                if (KIND == GDN) {
-#pragma unroll
-                    for (int e = 0; e < KPL; ++e) w[e] = fmaf(-bt * x, kf[e], w[e]);  // w^ -= b (k . w^) k
-                }
-                gsc *= at;
-            }
-        }
+        backward_chunk<KIND, DK, DV, QT>(ks, vs, as, nt, a_l, b_l, w, ob, gsc, lane);
         __syncwarp();  // every lane is done with the slots before the next chunk refills them
     }
     if (KIND != KDA) {
@@ -245,6 +259,188 @@ decode_step_kernel(const float *__restrict__ P, const float *__restrict__ R, con
     else *reinterpret_cast<float2 *>(oh) = make_float2(acc[0], acc[1]);
 }
 
+// ---------------------------------------------------------------------------
+// Persistent, pipelined decode step.  A warp owns a contiguous run of heads in
+// (h, b) order and keeps two shared-memory stages: while it computes head i from
+// one stage, head i+1's query row and its j buffered k, v (and KDA decay) rows
+// (contiguous blocks) land in the other by 16-byte cp.async copies, one commit
+// group per head, and head i+1's per-token scalars and first eight sketch columns
+// are in flight into registers.  The sketch columns stay in registers because
+// each lane reads whole sketch rows, which in shared memory would put every lane
+// of a warp on the same bank.  The coefficient rows R of the warp's head index h
+// stay in registers and are reloaded only when h changes.  The per-head
+// arithmetic is that of the kernel above.  Fewer warps fit per SM than for that
+// kernel (two stages, more registers), so the launcher takes this one only where
+// at least DEC_PERSIST_MIN_WARPS stay resident.
+// ---------------------------------------------------------------------------
+// A warp copies `bytes` (a multiple of 16) from global to shared memory in 16-byte
+// cp.async pieces (L2 only), lane-strided.
+__device__ __forceinline__ void copy16(char *dst, const void *src, int bytes, int lane) {
+    const char *s = static_cast<const char *>(src);
+    for (int i = lane * 16; i < bytes; i += 32 * 16)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dec_smem(dst + i)), "l"(s + i) : "memory");
+}
+
+template <int KIND, int DK, int DV, typename QT>
+struct DecStage {
+    static constexpr int QB = DK * (int)sizeof(QT);
+    using SL = DecSlots<KIND, DK, DV, QT>;
+    __host__ __device__ static int tokens(int j) { return j * (SL::KB + SL::VB + SL::AB); }
+    // query row, k rows, v rows, decay rows: each a multiple of 16 bytes
+    __host__ __device__ static int bytes(int j) { return QB + tokens(j); }
+};
+
+template <int KIND, int DK, int DV, typename QT>
+__global__ void __launch_bounds__(DEC_WARPS * 32)
+decode_step_persistent(const float *__restrict__ P, const float *__restrict__ R, const QT *__restrict__ qv,
+                       const QT *__restrict__ kbuf, const QT *__restrict__ vbuf,
+                       const float *__restrict__ abuf, const float *__restrict__ bbuf,
+                       float *__restrict__ o, int B, int H, int r, int j, int W) {
+    using SL = DecSlots<KIND, DK, DV, QT>;
+    using STG = DecStage<KIND, DK, DV, QT>;
+    constexpr int KPL = DK / 32, VPL = DV / 32;
+    extern __shared__ __align__(16) char smem[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int NH = B * H;
+    const int sbytes = STG::bytes(j);
+    char *const stage0 = smem + (size_t)warp * 2 * sbytes;
+
+    // this warp's run of heads (flat (h, b) order index i; head = b * H + h)
+    const int GW = gridDim.x * DEC_WARPS;
+    const int per = (NH + GW - 1) / GW;
+    const int i0 = (blockIdx.x * DEC_WARPS + warp) * per;
+    const int i1 = min(NH, i0 + per);
+    if (i0 >= i1) return;  // the whole warp; the kernel has no CTA-wide barrier
+
+    // every lane starts its share of the 16-byte copies of one head into stage s (one commit group)
+    auto issue = [&](int head, int s) {
+        char *sb = stage0 + s * sbytes;
+        char *qs = sb, *ks = qs + STG::QB, *vs = ks + j * SL::KB, *as = vs + j * SL::VB;
+        copy16(qs, qv + (size_t)head * DK, STG::QB, lane);
+        copy16(ks, kbuf + (size_t)head * W * DK, j * SL::KB, lane);
+        copy16(vs, vbuf + (size_t)head * W * DV, j * SL::VB, lane);
+        if (KIND == KDA) copy16(as, abuf + (size_t)head * W * DK, j * SL::AB, lane);
+        asm volatile("cp.async.commit_group;\n" ::: "memory");
+    };
+    // every lane: the per-token scalars of one head (token t in lane t, j <= 32) and the first
+    // DEC_RPRE sketch columns of the lane's value channels, into registers
+    auto scalars = [&](int head, float &al, float &bl, float (&pp)[VPL][DEC_RPRE]) {
+        al = (KIND != KDA && lane < j) ? abuf[(size_t)head * W + lane] : 1.f;
+        bl = (KIND != MAMBA2 && lane < j) ? bbuf[(size_t)head * W + lane] : 1.f;
+        const float *Ph = P + (size_t)head * DV * r;
+#pragma unroll
+        for (int e = 0; e < VPL; ++e) {
+            const float *row = Ph + (size_t)(lane * VPL + e) * r;
+            if ((r & 3) == 0 && r >= DEC_RPRE) {
+                const float4 a = *reinterpret_cast<const float4 *>(row), b = *reinterpret_cast<const float4 *>(row + 4);
+                pp[e][0] = a.x; pp[e][1] = a.y; pp[e][2] = a.z; pp[e][3] = a.w;
+                pp[e][4] = b.x; pp[e][5] = b.y; pp[e][6] = b.z; pp[e][7] = b.w;
+            } else {
+#pragma unroll
+                for (int m = 0; m < DEC_RPRE; ++m) pp[e][m] = m < r ? row[m] : 0.f;
+            }
+        }
+    };
+
+    int nh = i0 / B, nb = i0 - nh * B;  // the next head to issue
+    int ch = nh, cb = nb;               // the head being computed
+    float a_c, b_c, a_n = 1.f, b_n = 1.f, pp_c[VPL][DEC_RPRE], pp_n[VPL][DEC_RPRE];
+    issue(nb * H + nh, 0);
+    scalars(nb * H + nh, a_c, b_c, pp_c);
+    if (++nb == B) { nb = 0; ++nh; }
+
+    int h_rows = -1;
+    float rr[DEC_RPRE][KPL];
+    for (int i = i0, it = 0; i < i1; ++i, ++it) {
+        const int s = it & 1;
+        const int head = cb * H + ch;
+        const bool more = i + 1 < i1;
+        if (more) {
+            issue(nb * H + nh, s ^ 1);
+            scalars(nb * H + nh, a_n, b_n, pp_n);
+            if (++nb == B) { nb = 0; ++nh; }
+        }
+        const float *Rh = R + (size_t)ch * r * DK;
+        if (ch != h_rows) {  // warp-uniform
+#pragma unroll
+            for (int m = 0; m < DEC_RPRE; ++m) {
+                if (m < r) load_n<KPL>(Rh + (size_t)m * DK + lane * KPL, rr[m]);
+                else {
+#pragma unroll
+                    for (int e = 0; e < KPL; ++e) rr[m][e] = 0.f;
+                }
+            }
+            h_rows = ch;
+        }
+        // this head's group has landed (the next head's may still be in flight); the warp
+        // barrier makes every lane's copies visible to the whole warp
+        if (more) asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+        else asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+        __syncwarp();
+        const char *sb = stage0 + s * sbytes;
+        const char *qs = sb, *ks = qs + STG::QB, *vs = ks + j * SL::KB, *as = vs + j * SL::VB;
+
+        float acc[VPL];
+        float w[KPL], ob[VPL];
+        load_n<KPL>(reinterpret_cast<const QT *>(qs) + lane * KPL, w);
+#pragma unroll
+        for (int e = 0; e < VPL; ++e) ob[e] = 0.f;
+        float gsc = 1.f;
+        backward_chunk<KIND, DK, DV, QT>(ks, vs, as, j, a_c, b_c, w, ob, gsc, lane);
+        if (KIND != KDA) {
+#pragma unroll
+            for (int e = 0; e < KPL; ++e) w[e] *= gsc;
+        }
+
+        // c = R q~ (eight rows per warp all-reduce; rows past the first eight from L1/L2),
+        // o = P c + o_buf (the first eight sketch columns from registers, the rest from L1/L2)
+        const float *Ph = P + (size_t)head * DV * r;
+#pragma unroll
+        for (int e = 0; e < VPL; ++e) acc[e] = ob[e];
+#pragma unroll 1
+        for (int m0 = 0; m0 < r; m0 += DEC_RPRE) {
+            float c[DEC_RPRE];
+#pragma unroll
+            for (int mm = 0; mm < DEC_RPRE; ++mm) {
+                c[mm] = 0.f;
+                if (m0 == 0) {
+#pragma unroll
+                    for (int e = 0; e < KPL; ++e) c[mm] = fmaf(rr[mm][e], w[e], c[mm]);
+                } else if (m0 + mm < r) {
+                    float rv[KPL];
+                    load_n<KPL>(Rh + (size_t)(m0 + mm) * DK + lane * KPL, rv);
+#pragma unroll
+                    for (int e = 0; e < KPL; ++e) c[mm] = fmaf(rv[e], w[e], c[mm]);
+                }
+            }
+            warp_allreduce8(c, lane);
+#pragma unroll
+            for (int mm = 0; mm < DEC_RPRE; ++mm) {
+                if (m0 == 0) {
+#pragma unroll
+                    for (int e = 0; e < VPL; ++e) acc[e] = fmaf(pp_c[e][mm], c[mm], acc[e]);
+                } else if (m0 + mm < r) {
+#pragma unroll
+                    for (int e = 0; e < VPL; ++e)
+                        acc[e] = fmaf(Ph[(size_t)(lane * VPL + e) * r + m0 + mm], c[mm], acc[e]);
+                }
+            }
+        }
+        float *oh = o + (size_t)head * DV + lane * VPL;
+        if constexpr (VPL == 4) *reinterpret_cast<float4 *>(oh) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        else *reinterpret_cast<float2 *>(oh) = make_float2(acc[0], acc[1]);
+
+        __syncwarp();  // every lane is done with this stage before it is refilled
+        a_c = a_n;
+        b_c = b_n;
+#pragma unroll
+        for (int e = 0; e < VPL; ++e)
+#pragma unroll
+            for (int m = 0; m < DEC_RPRE; ++m) pp_c[e][m] = pp_n[e][m];
+        if (++cb == B) { cb = 0; ++ch; }
+    }
+}
+
 int launch_decode_step(const sketchssm_dims &d, const float *P, const float *R, const void *q,
                        const void *k, const void *v, const float *alpha, const float *beta, int j,
                        float *o, cudaStream_t stream) {
@@ -256,6 +452,31 @@ int launch_decode_step(const sketchssm_dims &d, const float *P, const float *R, 
         const int grid = (NH + DEC_WARPS - 1) / DEC_WARPS;
         auto go = [&](auto DVc) -> int {
             constexpr int DV = decltype(DVc)::value;
+            // the persistent pipelined kernel, when a warp's two stages leave enough warps per SM
+            if (j <= 32) {
+                const size_t psmem = (size_t)DEC_WARPS * 2 * DecStage<KIND, DK, DV, QT>::bytes(j);
+                if (psmem <= 227 * 1024) {
+                    auto pk = decode_step_persistent<KIND, DK, DV, QT>;
+                    static bool p_opted_in = false;
+                    if (!p_opted_in) {
+                        if (cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+                            cudaSuccess)
+                            return SKSSM_ERR_CUDA;
+                        p_opted_in = true;
+                    }
+                    int sms = 0, per_sm = 0;
+                    if (sm_count(&sms) != SKSSM_OK ||
+                        blocks_per_sm(reinterpret_cast<const void *>(pk), DEC_WARPS * 32, psmem, &per_sm) != SKSSM_OK)
+                        return SKSSM_ERR_CUDA;
+                    if (per_sm * DEC_WARPS >= DEC_PERSIST_MIN_WARPS) {
+                        const int pgrid = grid < sms * per_sm ? grid : sms * per_sm;
+                        pk<<<pgrid, DEC_WARPS * 32, psmem, stream>>>(
+                            P, R, static_cast<const QT *>(q), static_cast<const QT *>(k), static_cast<const QT *>(v),
+                            alpha, beta, o, d.B, d.H, d.r, j, d.W);
+                        return launch_status();
+                    }
+                }
+            }
             // tokens per bulk round trip (<= 32: one per lane); KDA rows are twice as wide, and fewer
             // of them per trip keep more warps resident
             const int jmax = KIND == KDA ? 8 : 32;

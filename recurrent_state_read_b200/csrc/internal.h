@@ -49,6 +49,44 @@ int launch_update_window(const sketchssm_dims &d, void *S, float *P, const float
 int update_wait_giveups(bool reset, unsigned *count);
 int decode_wait_giveups(bool reset, unsigned *count);
 
+// Resident CTAs per SM of a kernel at this block size and dynamic shared memory.
+// The occupancy query costs host time comparable to a short kernel, so results are
+// cached per calling thread (a few entries, replaced round-robin).
+inline int blocks_per_sm(const void *kern, int threads, size_t smem, int *per_sm) {
+    struct Entry {
+        const void *fn;
+        int threads;
+        size_t smem;
+        int per;
+    };
+    thread_local Entry cache[8] = {};
+    thread_local int next = 0;
+    for (const Entry &e : cache)
+        if (e.fn == kern && e.threads == threads && e.smem == smem) {
+            *per_sm = e.per;
+            return SKSSM_OK;
+        }
+    int per = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, kern, threads, smem) != cudaSuccess) return SKSSM_ERR_CUDA;
+    cache[next] = Entry{kern, threads, smem, per};
+    next = (next + 1) & 7;
+    *per_sm = per;
+    return SKSSM_OK;
+}
+
+// SM count of the current device, cached per calling thread and device.
+inline int sm_count(int *sms) {
+    thread_local int dev_cached = -1, count = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SKSSM_ERR_CUDA;
+    if (dev != dev_cached) {
+        if (cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return SKSSM_ERR_CUDA;
+        dev_cached = dev;
+    }
+    *sms = count;
+    return SKSSM_OK;
+}
+
 // Read (and optionally clear) a __device__ counter from the host.
 template <typename T>
 inline int read_counter(const T *symbol, bool reset, unsigned *count) {

@@ -516,10 +516,9 @@ int launch_update_window(const sketchssm_dims &d, void *S, float *P, const float
                     return SKSSM_ERR_CUDA;
                 opted_in = true;
             }
-            int dev = 0, sms = 0, per_sm = 0;
-            if (cudaGetDevice(&dev) != cudaSuccess ||
-                cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, L.total) != cudaSuccess)
+            int sms = 0, per_sm = 0;
+            if (sm_count(&sms) != SKSSM_OK ||
+                blocks_per_sm(reinterpret_cast<const void *>(kern), threads, L.total, &per_sm) != SKSSM_OK)
                 return SKSSM_ERR_CUDA;
             if (per_sm >= 1) {
                 const int grid = NH < sms * per_sm ? NH : sms * per_sm;

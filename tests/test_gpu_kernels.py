@@ -172,6 +172,33 @@ def test_update_window_many_heads_per_cta(kind):
         assert state_err(P.reshape(B * H, dv, r).double().cpu().numpy(), Pref) <= STATE_TOL, n
 
 
+@pytest.mark.parametrize("kind", ["mamba2", "gdn", "kda"])
+def test_decode_step_many_heads_per_warp(kind):
+    """6400 heads (B=16, H=400): the pipelined decode step runs several heads per warp, across
+    changes of h (new coefficient rows) inside one warp's run; every head is checked."""
+    import recurrent_state_read_b200 as rs
+
+    dk = dv = 64
+    r, W = 8, 8
+    cfg, d, S0, U, R, tok = _setup(kind, dk, dv, r, W, torch.float32, torch.bfloat16, B=16, H=400, seed=4)
+    B, H = d.B, d.H
+    g = torch.Generator().manual_seed(9)
+    P = torch.randn(B, H, dv, r, generator=g)
+    ft = flat_tokens(tok)
+    dev = to_device(tok)
+    win = to_window(dev)
+    Rh = oracle.per_head(R, H, np.arange(B * H))
+    for j in (1, 5, W):
+        o = torch.full((B, H, dv), float("nan"), device="cuda")
+        rs.sketchssm_decode_step(d, P.cuda(), R.cuda(), dev["q"][j - 1], win["k"], win["v"], win["alpha"],
+                                 win["beta"], j, o)
+        torch.cuda.synchronize()
+        sl = slice(0, j)
+        ref = oracle.sketch_read(kind, P.reshape(B * H, dv, r), Rh, ft["q"][j - 1], ft["k"][sl], ft["v"][sl],
+                                 ft["alpha"][sl], None if ft["beta"] is None else ft["beta"][sl])
+        assert rel_l2(o.reshape(B * H, dv).cpu(), ref) <= TIGHT_OUT, j
+
+
 def test_complete_basis_sketch_is_exact_read():
     """r = dk with U = R = I: decode-step outputs equal the full-read outputs (GPU both sides)."""
     import recurrent_state_read_b200 as rs

@@ -101,8 +101,9 @@ int sketchssm_version(void);
  * state_dtype, nearest-even, for SKSSM_BF16); then write P = S_stored^T U.
  * n_tokens = 0 is a sketch refresh only (S is read, not written).
  *   S        in/out [B][H][dv][dk] state_dtype
- *   P        out    [B][H][dv][r] fp32
- *   U        in     [H][r][dk] fp32 (basis rows)
+ *   P        out    [B][H][dv][r] fp32; NULL: no sketch refresh (a plain buffered
+ *            state update, the window-end write of the ReplaySSM-style path)
+ *   U        in     [H][r][dk] fp32 (basis rows); may be NULL when P is
  *   k, v, alpha, beta  in: window buffer slots 0..n_tokens-1 (NULL allowed when
  *            n_tokens == 0; beta NULL allowed for SKSSM_MAMBA2)
  * Errors: ERR_NULL, ERR_DIMS, ERR_DTYPE, ERR_RANGE (n_tokens < 0 or > W),
@@ -111,6 +112,24 @@ int sketchssm_version(void);
 int sketchssm_update_window(const sketchssm_dims *dims, void *S, float *P, const float *U,
                             const void *k, const void *v, const float *alpha, const float *beta,
                             int n_tokens, void *stream);
+
+/*
+ * sketchssm_update_window_read -- the window update with the exact read of the
+ * window's last step fused in.  The update already holds every head's updated
+ * state on chip (SketchSSM abstract: one full-state read per state update), so
+ * the read of the step whose token is the last one applied, o = S^T q, costs no
+ * state traffic; that step then needs no sketch read and has no approximation
+ * error.  Everything sketchssm_update_window does, plus, per head:
+ *     o = S_n^T q   from the updated state in fp32, before the storage rounding
+ *                   (as the full-read step reads it)
+ *   q   in  [B][H][dk] qkv_dtype, the query of the step whose token is slot n_tokens-1
+ *   o   out [B][H][dv] fp32
+ * n_tokens = 0 reads the unchanged state.
+ * Errors: as sketchssm_update_window, and ERR_NULL / ERR_ALIGN for q and o.
+ */
+int sketchssm_update_window_read(const sketchssm_dims *dims, void *S, float *P, const float *U,
+                                 const void *k, const void *v, const float *alpha, const float *beta,
+                                 int n_tokens, const void *q, float *o, void *stream);
 
 /*
  * sketchssm_decode_step -- one decode step inside a window, reading only the sketch.
@@ -148,6 +167,25 @@ int sketchssm_decode_step(const sketchssm_dims *dims, const float *P, const floa
 int sketchssm_fullread_decode(const sketchssm_dims *dims, void *S, const void *q, const void *k,
                               const void *v, const float *alpha, const float *beta, float *o,
                               void *stream);
+
+/*
+ * sketchssm_replay_decode_step -- the second baseline: one decode step of a
+ * buffered window that reads the full window-start state (ReplaySSM, as the
+ * SketchSSM abstract and the digest bullet "Background" describe it: updates are
+ * buffered and the state is written once per window, but every query still
+ * reads the full state).  Per head, with the backward pass of
+ * sketchssm_decode_step:  o = S^T q~ + o_buf  -- the exact read of step j.
+ * S is read, not written; the window ends with sketchssm_update_window (P may be
+ * NULL there).
+ *   S   in [B][H][dv][dk] state_dtype, the window-start state
+ *   q   in [B][H][dk];  k, v, alpha, beta in: window buffer slots 0..j-1
+ *   o   out [B][H][dv] fp32
+ * Errors: ERR_NULL, ERR_DIMS, ERR_DTYPE, ERR_RANGE (j < 1 or j > W), ERR_ALIGN,
+ * ERR_CUDA.
+ */
+int sketchssm_replay_decode_step(const sketchssm_dims *dims, const void *S, const void *q, const void *k,
+                                 const void *v, const float *alpha, const float *beta, int j, float *o,
+                                 void *stream);
 
 /*
  * sketchssm_device_error_count -- kernels never wait without bound: the decode

@@ -31,8 +31,10 @@ EXPORTS = (
     "sketchssm_status_string",
     "sketchssm_version",
     "sketchssm_update_window",
+    "sketchssm_update_window_read",
     "sketchssm_decode_step",
     "sketchssm_fullread_decode",
+    "sketchssm_replay_decode_step",
     "sketchssm_calibrate_workspace_bytes",
     "sketchssm_calibrate_basis",
     "sketchssm_calibrate_basis_noalloc",
@@ -73,8 +75,10 @@ def library() -> ctypes.CDLL:
         lib.sketchssm_version.argtypes = []
         lib.sketchssm_version.restype = i
         lib.sketchssm_update_window.argtypes = [D, P, P, P, P, P, P, P, i, P]
+        lib.sketchssm_update_window_read.argtypes = [D, P, P, P, P, P, P, P, i, P, P, P]
         lib.sketchssm_decode_step.argtypes = [D, P, P, P, P, P, P, P, i, P, P]
         lib.sketchssm_fullread_decode.argtypes = [D, P, P, P, P, P, P, P, P]
+        lib.sketchssm_replay_decode_step.argtypes = [D, P, P, P, P, P, P, i, P, P]
         lib.sketchssm_calibrate_workspace_bytes.argtypes = [D, i, i]
         lib.sketchssm_calibrate_workspace_bytes.restype = ctypes.c_size_t
         lib.sketchssm_calibrate_basis.argtypes = [D, P, i, P, i, ctypes.c_double, P, P, P,
@@ -82,7 +86,8 @@ def library() -> ctypes.CDLL:
         lib.sketchssm_calibrate_basis_noalloc.argtypes = [D, P, i, P, i, ctypes.c_double, P, P, P]
         lib.sketchssm_device_error_count.argtypes = [i]
         lib.sketchssm_device_error_count.restype = i
-        for f in ("sketchssm_update_window", "sketchssm_decode_step", "sketchssm_fullread_decode",
+        for f in ("sketchssm_update_window", "sketchssm_update_window_read", "sketchssm_decode_step",
+                  "sketchssm_replay_decode_step", "sketchssm_fullread_decode",
                   "sketchssm_calibrate_basis", "sketchssm_calibrate_basis_noalloc"):
             getattr(lib, f).restype = i
         _lib = lib
@@ -137,14 +142,31 @@ def _token_ptrs(d: sketchssm_dims, slots: int, k, v, alpha, beta):
 
 
 def sketchssm_update_window(d: sketchssm_dims, S, P, U, k, v, alpha, beta, n_tokens: int, stream=None):
-    """Apply window-buffer tokens 0..n_tokens-1 to S exactly and refresh P = S^T U (one kernel)."""
+    """Apply window-buffer tokens 0..n_tokens-1 to S exactly and refresh P = S^T U (one kernel).
+    P = None (and U = None): no sketch refresh."""
     NH = d.B * d.H
-    args = (_ptr(S, "S", NH * d.dv * d.dk, _dt(d.state_dtype)), _ptr(P, "P", NH * d.dv * d.r, torch.float32),
-            _ptr(U, "U", d.H * d.dk * d.r, torch.float32))
+    args = (_ptr(S, "S", NH * d.dv * d.dk, _dt(d.state_dtype)),
+            None if P is None else _ptr(P, "P", NH * d.dv * d.r, torch.float32),
+            None if U is None else _ptr(U, "U", d.H * d.dk * d.r, torch.float32))
     toks = _token_ptrs(d, d.W, k, v, alpha, beta) if n_tokens > 0 else (None,) * 4
     _check("sketchssm_update_window",
            library().sketchssm_update_window(ctypes.byref(d), *args, *toks, int(n_tokens),
                                              ctypes.c_void_p(_stream(stream))))
+
+
+def sketchssm_update_window_read(d: sketchssm_dims, S, P, U, k, v, alpha, beta, n_tokens: int, q, o,
+                                 stream=None):
+    """sketchssm_update_window plus the exact read o = S^T q of the step whose token is the last
+    one applied (q [B,H,dk] qkv dtype, o [B,H,dv] fp32), in the same kernel."""
+    NH = d.B * d.H
+    args = (_ptr(S, "S", NH * d.dv * d.dk, _dt(d.state_dtype)), _ptr(P, "P", NH * d.dv * d.r, torch.float32),
+            _ptr(U, "U", d.H * d.dk * d.r, torch.float32))
+    toks = _token_ptrs(d, d.W, k, v, alpha, beta) if n_tokens > 0 else (None,) * 4
+    _check("sketchssm_update_window_read",
+           library().sketchssm_update_window_read(ctypes.byref(d), *args, *toks, int(n_tokens),
+                                                  _ptr(q, "q", NH * d.dk, _dt(d.qkv_dtype)),
+                                                  _ptr(o, "o", NH * d.dv, torch.float32),
+                                                  ctypes.c_void_p(_stream(stream))))
 
 
 def sketchssm_decode_step(d: sketchssm_dims, P, R, q, k, v, alpha, beta, j: int, o, stream=None):
@@ -155,6 +177,17 @@ def sketchssm_decode_step(d: sketchssm_dims, P, R, q, k, v, alpha, beta, j: int,
         ctypes.byref(d), _ptr(P, "P", NH * d.dv * d.r, torch.float32),
         _ptr(R, "R", d.H * d.r * d.dk, torch.float32), _ptr(q, "q", NH * d.dk, _dt(d.qkv_dtype)),
         *toks, int(j), _ptr(o, "o", NH * d.dv, torch.float32), ctypes.c_void_p(_stream(stream))))
+
+
+def sketchssm_replay_decode_step(d: sketchssm_dims, S, q, k, v, alpha, beta, j: int, o, stream=None):
+    """ReplaySSM-style decode step j: the exact read o = S^T q~ + o_buf of the window-start state S
+    (read, not written) and window-buffer tokens 0..j-1."""
+    NH = d.B * d.H
+    toks = _token_ptrs(d, d.W, k, v, alpha, beta)
+    _check("sketchssm_replay_decode_step", library().sketchssm_replay_decode_step(
+        ctypes.byref(d), _ptr(S, "S", NH * d.dv * d.dk, _dt(d.state_dtype)),
+        _ptr(q, "q", NH * d.dk, _dt(d.qkv_dtype)), *toks, int(j), _ptr(o, "o", NH * d.dv, torch.float32),
+        ctypes.c_void_p(_stream(stream))))
 
 
 def sketchssm_fullread_decode(d: sketchssm_dims, S, q, k, v, alpha, beta, o, stream=None):

@@ -62,11 +62,25 @@ int sketchssm_update_window(const sketchssm_dims *d, void *S, float *P, const fl
                             void *stream) {
     int rc = check_dims(d);
     if (rc) return rc;
-    if (!S || !P || !U) return SKSSM_ERR_NULL;
+    if (!S || (P && !U)) return SKSSM_ERR_NULL;  // P == NULL: a state update without a sketch refresh
     if (n_tokens < 0 || n_tokens > d->W) return SKSSM_ERR_RANGE;
     if (n_tokens > 0 && (rc = check_tokens(d, k, v, alpha, beta))) return rc;
     if (!aligned(S, 16) || !aligned(P, 16) || !aligned(U, 16)) return SKSSM_ERR_ALIGN;
-    return launch_update_window(*d, S, P, U, k, v, alpha, beta, n_tokens, (cudaStream_t)stream);
+    return launch_update_window(*d, S, P, P ? U : nullptr, k, v, alpha, beta, n_tokens, nullptr, nullptr,
+                                (cudaStream_t)stream);
+}
+
+int sketchssm_update_window_read(const sketchssm_dims *d, void *S, float *P, const float *U, const void *k,
+                                            const void *v, const float *alpha, const float *beta, int n_tokens,
+                                            const void *q, float *o, void *stream) {
+    int rc = check_dims(d);
+    if (rc) return rc;
+    if (!S || !P || !U || !q || !o) return SKSSM_ERR_NULL;
+    if (n_tokens < 0 || n_tokens > d->W) return SKSSM_ERR_RANGE;
+    if (n_tokens > 0 && (rc = check_tokens(d, k, v, alpha, beta))) return rc;
+    if (!aligned(S, 16) || !aligned(P, 16) || !aligned(U, 16) || !aligned(q, 16) || !aligned(o, 16))
+        return SKSSM_ERR_ALIGN;
+    return launch_update_window(*d, S, P, U, k, v, alpha, beta, n_tokens, q, o, (cudaStream_t)stream);
 }
 
 int sketchssm_decode_step(const sketchssm_dims *d, const float *P, const float *R, const void *q,
@@ -90,6 +104,17 @@ int sketchssm_fullread_decode(const sketchssm_dims *d, void *S, const void *q, c
     if ((rc = check_tokens(d, k, v, alpha, beta))) return rc;
     if (!aligned(S, 16) || !aligned(q, 16) || !aligned(o, 16)) return SKSSM_ERR_ALIGN;
     return launch_fullread(*d, S, q, k, v, alpha, beta, o, (cudaStream_t)stream);
+}
+
+int sketchssm_replay_decode_step(const sketchssm_dims *d, const void *S, const void *q, const void *k, const void *v,
+                                 const float *alpha, const float *beta, int j, float *o, void *stream) {
+    int rc = check_dims(d);
+    if (rc) return rc;
+    if (!S || !q || !o) return SKSSM_ERR_NULL;
+    if (j < 1 || j > d->W) return SKSSM_ERR_RANGE;
+    if ((rc = check_tokens(d, k, v, alpha, beta))) return rc;
+    if (!aligned(S, 16) || !aligned(q, 16) || !aligned(o, 16)) return SKSSM_ERR_ALIGN;
+    return launch_replay_decode(*d, S, q, k, v, alpha, beta, j, o, (cudaStream_t)stream);
 }
 
 size_t sketchssm_calibrate_workspace_bytes(const sketchssm_dims *d, int Nq, int Ns) {

@@ -27,8 +27,7 @@
 // are in flight: 64 registers per thread keep eight 4-warp CTAs on an SM.  The
 // wait on the copies is bounded: a give-up is counted in a device flag
 // (sketchssm_device_error_count) and the warp returns.
-#include "internal.h"
-#include "state_tile.cuh"
+#include "decode_common.cuh"
 
 namespace skssm {
 
@@ -59,90 +58,6 @@ __device__ __forceinline__ void dec_bulk(void *dst, const void *src, int bytes, 
                      dec_smem(dst)),
                  "l"(src), "r"(bytes), "r"(dec_smem(bar))
                  : "memory");
-}
-
-// Per-warp shared memory: barrier (16 B), then jc slots of k rows, v rows, (KDA) decay rows.
-template <int KIND, int DK, int DV, typename QT>
-struct DecSlots {
-    static constexpr int KB = DK * (int)sizeof(QT), VB = DV * (int)sizeof(QT);
-    static constexpr int AB = KIND == KDA ? DK * 4 : 0;
-    __host__ __device__ static int bytes(int jc) { return 16 + jc * (KB + VB + AB); }
-};
-
-template <int N, typename T>
-__device__ __forceinline__ void load_n(const T *p, float *out) {
-    if constexpr (N == 4) load4(p, out);
-    else load2(p, out);
-}
-
-// The backward pass over one chunk of buffered tokens held in shared memory
-// (slots 0 .. nt-1, oldest first; ks/vs/as their k, v and KDA decay rows), newest
-// first: per token x = k . w, o_buf += b x v, w <- M^T w.  Lane t holds the chunk's
-// token-t scalars a_l, b_l.  For scalar decay w is kept as gsc * w^.
-template <int KIND, int DK, int DV, typename QT>
-__device__ __forceinline__ void backward_chunk(const char *ks, const char *vs, const char *as, int nt, float a_l,
-                                               float b_l, float (&w)[DK / 32], float (&ob)[DV / 32], float &gsc,
-                                               int lane) {
-    using SL = DecSlots<KIND, DK, DV, QT>;
-    constexpr int KPL = DK / 32, VPL = DV / 32;
-    if constexpr (KIND == MAMBA2) {
-        // w stays q: the dots of eight tokens are independent and share one warp all-reduce
-        for (int t0 = nt - 1; t0 >= 0; t0 -= 8) {
-            float x[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                x[u] = 0.f;
-                if (t0 - u >= 0) {
-                    float kf[KPL];
-                    load_n<KPL>(reinterpret_cast<const QT *>(ks + (t0 - u) * SL::KB) + lane * KPL, kf);
-#pragma unroll
-                    for (int e = 0; e < KPL; ++e) x[u] = fmaf(kf[e], w[e], x[u]);
-                }
-            }
-            warp_allreduce8(x, lane);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                if (t0 - u >= 0) {  // warp-uniform
-                    const int sl = t0 - u;
-                    float vf[VPL];
-                    load_n<VPL>(reinterpret_cast<const QT *>(vs + sl * SL::VB) + lane * VPL, vf);
-                    const float s = gsc * x[u];  // (k . q) times the decay of the later tokens
-#pragma unroll
-                    for (int e = 0; e < VPL; ++e) ob[e] = fmaf(s, vf[e], ob[e]);
-                    gsc *= __shfl_sync(FULL, a_l, sl);
-                }
-            }
-        }
-    } else {
-        for (int sl = nt - 1; sl >= 0; --sl) {
-            float kf[KPL], vf[VPL];
-            load_n<KPL>(reinterpret_cast<const QT *>(ks + sl * SL::KB) + lane * KPL, kf);
-            load_n<VPL>(reinterpret_cast<const QT *>(vs + sl * SL::VB) + lane * VPL, vf);
-            const float at = __shfl_sync(FULL, a_l, sl), bt = __shfl_sync(FULL, b_l, sl);
-            float x = 0.f;
-#pragma unroll
-            for (int e = 0; e < KPL; ++e) x = fmaf(kf[e], w[e], x);
-            x = warp_sum(x);  // k . w (k . w^ for scalar decay)
-            if (KIND == KDA) {
-                const float s = bt * x;
-#pragma unroll
-                for (int e = 0; e < VPL; ++e) ob[e] = fmaf(s, vf[e], ob[e]);
-                float a[KPL];
-                load_n<KPL>(reinterpret_cast<const float *>(as + sl * SL::AB) + lane * KPL, a);
-#pragma unroll
-                for (int e = 0; e < KPL; ++e) w[e] = a[e] * fmaf(-s, kf[e], w[e]);
-            } else {
-                const float s = bt * gsc * x;  // b (k . w), w = gsc w^
-#pragma unroll
-                for (int e = 0; e < VPL; ++e) ob[e] = fmaf(s, vf[e], ob[e]);
-                if (KIND == GDN) {
-#pragma unroll
-                    for (int e = 0; e < KPL; ++e) w[e] = fmaf(-bt * x, kf[e], w[e]);  // w^ -= b (k . w^) k
-                }
-                gsc *= at;
-            }
-        }
-    }
 }
 
 template <int KIND, int DK, int DV, typename QT>

@@ -43,7 +43,7 @@ inline int launch_status() {
 }
 
 int launch_update_window(const sketchssm_dims &d, void *S, float *P, const float *U, const void *k,
-                         const void *v, const float *alpha, const float *beta, int n_tokens,
+                         const void *v, const float *alpha, const float *beta, int n_tokens, const void *q, float *o,
                          cudaStream_t stream);
 // Counts of bounded in-kernel waits that gave up (window update, decode step); reset clears them.
 int update_wait_giveups(bool reset, unsigned *count);
@@ -98,6 +98,8 @@ inline int read_counter(const T *symbol, bool reset, unsigned *count) {
     }
     return SKSSM_OK;
 }
+int launch_replay_decode(const sketchssm_dims &d, const void *S, const void *q, const void *k, const void *v,
+                         const float *alpha, const float *beta, int j, float *o, cudaStream_t stream);
 int launch_fullread(const sketchssm_dims &d, void *S, const void *q, const void *k, const void *v,
                     const float *alpha, const float *beta, float *o, cudaStream_t stream);
 int launch_decode_step(const sketchssm_dims &d, const float *P, const float *R, const void *q,

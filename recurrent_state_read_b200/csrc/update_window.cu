@@ -84,8 +84,9 @@ __device__ __forceinline__ void stage_rows(const T *__restrict__ src, size_t row
 template <int KIND, int DK, typename ST, int NC>
 __device__ __forceinline__ void apply_store_refresh(float (&s)[NC][DK / 8], const float *sk, const float *su,
                                                     const float *sv, const float *sg, const float *sut,
-                                                    const float *ss2, ST *__restrict__ S, float *__restrict__ P,
-                                                    int head, int dv, int r, int n, int c0, int l, int lane) {
+                                                    const float *ss2, const float *sq, ST *__restrict__ S,
+                                                    float *__restrict__ P, float *__restrict__ o, int head, int dv,
+                                                    int r, int n, int c0, int l, int lane) {
     using TL = TileLayout<DK, ST>;
     constexpr int EPL = TL::EPL;
     const int cl = NC == 8 ? l : l >> 1;  // the column whose reduced values this lane holds
@@ -120,23 +121,43 @@ __device__ __forceinline__ void apply_store_refresh(float (&s)[NC][DK / 8], cons
         }
     }
 
-    // final scale, storage rounding, one store of the state
+    // final scale
     if (KIND != KDA) {
         const float gam = sg[0];
 #pragma unroll
         for (int cc = 0; cc < NC; ++cc)
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) s[cc][e] = as_stored<ST>(s[cc][e] * gam);
+            for (int e = 0; e < EPL; ++e) s[cc][e] *= gam;
     } else {
         float gv[EPL];
         lane_channels_smem<DK, ST>(sg, l, gv);
 #pragma unroll
         for (int cc = 0; cc < NC; ++cc)
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) s[cc][e] = as_stored<ST>(s[cc][e] * gv[e]);
+            for (int e = 0; e < EPL; ++e) s[cc][e] *= gv[e];
     }
+    // the exact read of the window's last step, o = S^T q, from the updated fp32 state (the
+    // full-read step reads before storage rounding too)
+    if (sq != nullptr) {
+        float qv[EPL];
+        lane_channels_smem<DK, ST>(sq, l, qv);
+        float d[NC];
+#pragma unroll
+        for (int cc = 0; cc < NC; ++cc) d[cc] = dot<EPL>(qv, s[cc]);
+        float x;
+        if constexpr (NC == 8) x = octet_reduce_scatter(d, lane);
+        else x = octet_reduce4(d, lane);
+        if (NC == 8 || (l & 1) == 0) o[(size_t)head * dv + c0 + cl] = x;
+    }
+    // storage rounding, one store of the state
+#pragma unroll
+    for (int cc = 0; cc < NC; ++cc)
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) s[cc][e] = as_stored<ST>(s[cc][e]);
     if (n > 0) store_tile<DK, ST, NC>(S + (size_t)head * dv * DK, c0, l, s);
 
+    // sketch refresh (skipped when P is NULL: a plain buffered state update)
+    if (P == nullptr) return;
     // sketch refresh P[c][m] = sum_i S[i][c] U[i][m] from the stored values: per
     //    basis row m one dot per column and one octet reduction, after which lane
     //    l holds P[c0 + cl][m]; four basis rows per pass bound the rows in flight
@@ -175,7 +196,8 @@ template <int KIND, int DK, typename ST, typename QT, int NC>
 __global__ void __launch_bounds__(256)
 update_window_kernel(ST *__restrict__ S, float *__restrict__ P, const float *__restrict__ U,
                      const QT *__restrict__ kbuf, const QT *__restrict__ vbuf,
-                     const float *__restrict__ abuf, const float *__restrict__ bbuf, int B, int H,
+                     const float *__restrict__ abuf, const float *__restrict__ bbuf,
+                     const QT *__restrict__ qv, float *__restrict__ o, int B, int H,
                      int dv, int r, int n, int W) {
     using TL = TileLayout<DK, ST>;
     constexpr int EPL = TL::EPL;
@@ -198,16 +220,19 @@ update_window_kernel(ST *__restrict__ S, float *__restrict__ P, const float *__r
     float *sut = sg + DK;                                  // [r][DK]: the head's basis rows
     float *ss1 = sut + (size_t)r * DK;                     // [n4]: b_t / g_t (Mamba-2: 1 / g_t)
     float *ss2 = ss1 + ((n + 3) & ~3);                     // [n4]: b_t
+    float *sq = ss2 + ((n + 3) & ~3);                      // [DK]: the last step's query (when read)
 
     // 1. the state goes in flight first, straight into registers
     float s[NC][EPL];
     load_tile<DK, ST, NC>(S + (size_t)head * dv * DK, c0, l, s);
 
     // 2. the basis rows, per-token scalars, then the tokens in fp32 with the scalars folded in
-    {
+    if (U != nullptr) {
         const float4 *src = reinterpret_cast<const float4 *>(U + (size_t)h * r * DK);
         for (int i = tid; i < r * DK / 4; i += nthr) reinterpret_cast<float4 *>(sut)[i] = src[i];
     }
+    if (qv != nullptr)
+        for (int i = tid; i < DK; i += nthr) sq[i] = ld1(qv + (size_t)head * DK + i);
     if (KIND != KDA) {
         if (warp == 0) {
             // g_t = a_1 ... a_t by a warp prefix product (n <= 64: two tokens per lane)
@@ -249,7 +274,8 @@ update_window_kernel(ST *__restrict__ S, float *__restrict__ P, const float *__r
     }
     __syncthreads();
 
-    apply_store_refresh<KIND, DK, ST, NC>(s, sk, su, sv, sg, sut, ss2, S, P, head, dv, r, n, c0, l, lane);
+    apply_store_refresh<KIND, DK, ST, NC>(s, sk, su, sv, sg, sut, ss2, qv ? sq : nullptr, S, P, o, head, dv, r, n,
+                                          c0, l, lane);
 }
 
 // ---------------------------------------------------------------------------
@@ -292,9 +318,9 @@ __host__ __device__ inline int up16(int x) { return (x + 15) & ~15; }
 
 // Byte offsets of the persistent kernel's shared memory (host and device agree).
 struct PerLayout {
-    int stage_bytes, st, kr, vr, ar;  // inside a stage: state, raw k, raw v, raw decay (KDA)
-    int stages;                       // first stage (NS stages follow, stage_bytes apart)
-    int sk, su, sv, sg, sut, ss2, total;
+    int stage_bytes, st, kr, vr, ar, qr;  // inside a stage: state, raw k, raw v, raw decay (KDA), raw query
+    int stages;                           // first stage (NS stages follow, stage_bytes apart)
+    int sk, su, sv, sg, sut, ss2, sq, total;
 };
 
 __host__ __device__ inline PerLayout per_layout(int kind, int DK, int dv, int r, int n, int sbytes, int qbytes,
@@ -305,6 +331,7 @@ __host__ __device__ inline PerLayout per_layout(int kind, int DK, int dv, int r,
     L.kr = t; t += up16(n * DK * qbytes);
     L.vr = t; t += up16(n * dv * qbytes);
     L.ar = t; t += kind == KDA ? up16(n * DK * 4) : 0;
+    L.qr = t; t += up16(DK * qbytes);
     L.stage_bytes = t;
     int off = 16 * 2;  // two mbarriers, 16 bytes apart
     L.stages = off; off += ns * t;
@@ -314,6 +341,7 @@ __host__ __device__ inline PerLayout per_layout(int kind, int DK, int dv, int r,
     L.sg = off; off += up16(DK * 4);
     L.sut = off; off += up16(r * DK * 4);
     L.ss2 = off; off += up16(n * 4);
+    L.sq = off; off += up16(DK * 4);
     L.total = off;
     return L;
 }
@@ -322,8 +350,9 @@ template <int KIND, int DK, typename ST, typename QT, int NC>
 __global__ void __launch_bounds__(256)
 update_window_persistent(ST *__restrict__ S, float *__restrict__ P, const float *__restrict__ U,
                          const QT *__restrict__ kbuf, const QT *__restrict__ vbuf,
-                         const float *__restrict__ abuf, const float *__restrict__ bbuf, int B, int H, int dv,
-                         int r, int n, int W, int ns) {
+                         const float *__restrict__ abuf, const float *__restrict__ bbuf,
+                         const QT *__restrict__ qv, float *__restrict__ o, int B, int H, int dv, int r, int n, int W,
+                         int ns) {
     using TL = TileLayout<DK, ST>;
     constexpr int EPL = TL::EPL;
     extern __shared__ __align__(128) float psm_f[];
@@ -347,9 +376,11 @@ update_window_persistent(ST *__restrict__ S, float *__restrict__ P, const float 
     float *sg = reinterpret_cast<float *>(smem + L.sg);
     float *sut = reinterpret_cast<float *>(smem + L.sut);
     float *ss2 = reinterpret_cast<float *>(smem + L.ss2);
+    float *sq = reinterpret_cast<float *>(smem + L.sq);
     const int state_bytes = dv * DK * (int)sizeof(ST);
     const int kbytes = n * DK * (int)sizeof(QT), vbytes = n * dv * (int)sizeof(QT);
     const int abytes = KIND == KDA ? n * DK * 4 : 0;
+    const int qbytes = qv != nullptr ? DK * (int)sizeof(QT) : 0;
 
     auto issue = [&](int w, int stage) {  // one thread
         char *sb = smem + L.stages + stage * L.stage_bytes;
@@ -357,9 +388,10 @@ update_window_persistent(ST *__restrict__ S, float *__restrict__ P, const float 
         uint64_t *bar = bars + 2 * stage;
         asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(upd_smem(bar)),
-                     "r"(state_bytes + kbytes + vbytes + abytes)
+                     "r"(state_bytes + kbytes + vbytes + abytes + qbytes)
                      : "memory");
         upd_bulk(sb + L.st, S + (size_t)head * dv * DK, state_bytes, bar);
+        if (qbytes) upd_bulk(sb + L.qr, qv + (size_t)head * DK, qbytes, bar);
         if (n > 0) {
             upd_bulk(sb + L.kr, kbuf + (size_t)head * W * DK, kbytes, bar);
             upd_bulk(sb + L.vr, vbuf + (size_t)head * W * dv, vbytes, bar);
@@ -419,10 +451,14 @@ update_window_persistent(ST *__restrict__ S, float *__restrict__ P, const float 
 #pragma unroll
             for (int q = 0; q < TL::NQ; ++q)
                 load16<ST>(st + (size_t)(c0 + cc) * DK + TL::chan(l, q, 0), &s[cc][q * TL::VEC]);
-        if (h != h_prev) {
+        if (h != h_prev && U != nullptr) {
             const float4 *src = reinterpret_cast<const float4 *>(U + (size_t)h * r * DK);
             for (int i = tid; i < r * DK / 4; i += nthr) reinterpret_cast<float4 *>(sut)[i] = src[i];
             h_prev = h;
+        }
+        if (qbytes) {
+            const QT *qr = reinterpret_cast<const QT *>(sb + L.qr);
+            for (int i = tid; i < DK; i += nthr) sq[i] = ld1(qr + i);
         }
         const QT *kr = reinterpret_cast<const QT *>(sb + L.kr);
         const QT *vr = reinterpret_cast<const QT *>(sb + L.vr);
@@ -484,19 +520,20 @@ update_window_persistent(ST *__restrict__ S, float *__restrict__ P, const float 
         __syncthreads();  // the stage is consumed; the fp32 staging is ready
         if (tid == 0 && w + ns < w_end) issue(w + ns, stage);
 
-        apply_store_refresh<KIND, DK, ST, NC>(s, sk, su, sv, sg, sut, ss2, S, P, head, dv, r, n, c0, l, lane);
+        apply_store_refresh<KIND, DK, ST, NC>(s, sk, su, sv, sg, sut, ss2, qbytes ? sq : nullptr, S, P, o, head, dv,
+                                              r, n, c0, l, lane);
     }
 }
 
 static size_t update_smem_bytes(const sketchssm_dims &d, int n) {
     const size_t n4 = (n + 3) & ~3;
     const size_t fl = (size_t)n * d.dk * (d.kind == SKSSM_KDA ? 2 : 1) + (size_t)n * d.dv + d.dk +
-                      (size_t)d.r * d.dk + 2 * n4;
+                      (size_t)d.r * d.dk + 2 * n4 + d.dk;
     return fl * sizeof(float);
 }
 
 int launch_update_window(const sketchssm_dims &d, void *S, float *P, const float *U, const void *k,
-                         const void *v, const float *alpha, const float *beta, int n,
+                         const void *v, const float *alpha, const float *beta, int n, const void *q, float *o,
                          cudaStream_t stream) {
     constexpr int LIMIT = 227 * 1024;
     return dispatch(d, [&](auto K, auto D, auto *sp, auto *qp) -> int {
@@ -523,8 +560,9 @@ int launch_update_window(const sketchssm_dims &d, void *S, float *P, const float
             if (per_sm >= 1) {
                 const int grid = NH < sms * per_sm ? NH : sms * per_sm;
                 kern<<<grid, threads, L.total, stream>>>(static_cast<ST *>(S), P, U, static_cast<const QT *>(k),
-                                                         static_cast<const QT *>(v), alpha, beta, d.B, d.H, d.dv,
-                                                         d.r, n, d.W, ns);
+                                                         static_cast<const QT *>(v), alpha, beta,
+                                                         static_cast<const QT *>(q), o, d.B, d.H, d.dv, d.r, n, d.W,
+                                                         ns);
                 return launch_status();
             }
         }
@@ -540,7 +578,8 @@ int launch_update_window(const sketchssm_dims &d, void *S, float *P, const float
             opted_in = true;
         }
         kern<<<NH, threads, smem, stream>>>(static_cast<ST *>(S), P, U, static_cast<const QT *>(k),
-                                            static_cast<const QT *>(v), alpha, beta, d.B, d.H, d.dv, d.r, n, d.W);
+                                            static_cast<const QT *>(v), alpha, beta, static_cast<const QT *>(q), o,
+                                            d.B, d.H, d.dv, d.r, n, d.W);
         return launch_status();
     });
 }

@@ -4,7 +4,9 @@ Timeline (SketchSSM abstract and the agihunt digest's "Mechanism details"):
 within a window of W steps the state is fixed; step j reads the sketch and the
 buffered tokens 1..j; after the window's last step one kernel applies the W
 buffered tokens to the state and refreshes the sketch.  The full-read baseline
-updates and reads the whole state at every step.  This module is host-side
+updates and reads the whole state at every step; the ReplaySSM-style baseline
+(the buffering the SketchSSM abstract starts from) reads the full window-start
+state at every step and writes it once per window.  This module is host-side
 control flow only: every arithmetic step runs in libsketchssm.so.
 """
 
@@ -15,8 +17,8 @@ from typing import Optional
 
 import torch
 
-from . import (sketchssm_decode_step, sketchssm_dims, sketchssm_fullread_decode,
-               sketchssm_update_window)
+from . import (sketchssm_decode_step, sketchssm_dims, sketchssm_fullread_decode, sketchssm_replay_decode_step,
+               sketchssm_update_window, sketchssm_update_window_read)
 
 
 @dataclasses.dataclass
@@ -56,14 +58,30 @@ class WindowBuffer:
 
 
 def sketch_window(d: sketchssm_dims, S, P, U, R, buf: WindowBuffer, out, n: Optional[int] = None,
-                  stream=None):
+                  stream=None, exact_last: bool = False):
     """One window of the sketch path: n decode steps (outputs into out[0..n-1], each [B,H,dv]
-    fp32) read the sketch; then one window update applies the n tokens and refreshes P."""
+    fp32) read the sketch; then one window update applies the n tokens and refreshes P.
+    exact_last: step n is not read from the sketch but exactly, inside the window update
+    (sketchssm_update_window_read), which holds the updated state anyway."""
     n = d.W if n is None else n
-    for j in range(1, n + 1):
+    for j in range(1, (n - 1 if exact_last else n) + 1):
         sketchssm_decode_step(d, P, R, buf.q[j - 1], buf.k, buf.v, buf.alpha, buf.beta, j, out[j - 1],
                               stream)
-    sketchssm_update_window(d, S, P, U, buf.k, buf.v, buf.alpha, buf.beta, n, stream)
+    if exact_last and n > 0:
+        sketchssm_update_window_read(d, S, P, U, buf.k, buf.v, buf.alpha, buf.beta, n, buf.q[n - 1],
+                                     out[n - 1], stream)
+    else:
+        sketchssm_update_window(d, S, P, U, buf.k, buf.v, buf.alpha, buf.beta, n, stream)
+
+
+def replay_window(d: sketchssm_dims, S, buf: WindowBuffer, out, n: Optional[int] = None, stream=None):
+    """One window of the ReplaySSM-style path: n decode steps each read the full window-start
+    state exactly (no write); one window update then applies the n tokens (no sketch)."""
+    n = d.W if n is None else n
+    for j in range(1, n + 1):
+        sketchssm_replay_decode_step(d, S, buf.q[j - 1], buf.k, buf.v, buf.alpha, buf.beta, j, out[j - 1],
+                                     stream)
+    sketchssm_update_window(d, S, None, None, buf.k, buf.v, buf.alpha, buf.beta, n, stream)
 
 
 def fullread_window(d: sketchssm_dims, S, tok: dict, out, n: Optional[int] = None, stream=None):

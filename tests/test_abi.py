@@ -84,10 +84,24 @@ def test_validation_codes(rs):
     bad = _d(rs)
     bad.state_dtype = 7
     assert uw(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, None) == -5
+    ur = lib.sketchssm_update_window_read
+    assert ur(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, None, FAKE, None) == -1  # q
+    assert ur(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, FAKE, None, None) == -1  # o
+    assert ur(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 17, FAKE, FAKE, None) == -3
+    assert ur(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, odd, FAKE, None) == -4
+    assert ur(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, FAKE, odd, None) == -4
+    assert ur(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, FAKE, FAKE, None) == -5
     ds = lib.sketchssm_decode_step
     assert ds(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, FAKE, None) == -3
     assert ds(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 17, FAKE, None) == -3
     assert ds(ctypes.byref(d), FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, 3, FAKE, None) == -1
+    rp = lib.sketchssm_replay_decode_step
+    assert rp(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, FAKE, None) == -3
+    assert rp(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 17, FAKE, None) == -3
+    assert rp(ctypes.byref(d), None, FAKE, FAKE, FAKE, FAKE, FAKE, 3, FAKE, None) == -1
+    assert rp(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, None, 3, FAKE, None) == -1  # GDN needs beta
+    assert rp(ctypes.byref(d), FAKE, odd, FAKE, FAKE, FAKE, FAKE, 3, FAKE, None) == -4
+    assert uw(ctypes.byref(d), FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, 4, None) == -1  # P without U
     fr = lib.sketchssm_fullread_decode
     assert fr(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, None) == -1
     assert fr(ctypes.byref(d), FAKE, FAKE, odd, FAKE, FAKE, FAKE, FAKE, None) == -4

@@ -96,6 +96,37 @@ def test_update_window(case):
 
 
 @pytest.mark.parametrize("case", CASES, ids=[_ids(c) for c in CASES])
+def test_update_window_read(case):
+    """The window update with the last step's exact read fused in: S and P as the plain update,
+    o = S_n^T q_n against the oracle's exact per-step read (before any storage rounding)."""
+    import recurrent_state_read_b200 as rs
+
+    kind, dk, dv, r, W, sdt, qdt = case
+    cfg, d, S0, U, R, tok = _setup(kind, dk, dv, r, W, sdt, qdt, seed=5)
+    B, H = d.B, d.H
+    Uh = oracle.per_head(U, H, np.arange(B * H))
+    ft = flat_tokens(tok)
+    dev = to_device(tok)
+    win = to_window(dev)
+    beta = lambda sl: None if ft["beta"] is None else ft["beta"][sl]
+    for n in sorted({1, max(1, W // 2), W}):
+        S = to_gpu_state(S0, B, H, sdt)
+        P = torch.full((B, H, dv, r), float("nan"), device="cuda")
+        o = torch.full((B, H, dv), float("nan"), device="cuda")
+        rs.sketchssm_update_window_read(d, S, P, U.transpose(1, 2).contiguous().cuda(), win["k"], win["v"],
+                                        win["alpha"], win["beta"], n, dev["q"][n - 1], o)
+        torch.cuda.synchronize()
+        sl = slice(0, n)
+        Sref, Pref = oracle.update_window(kind, S0, Uh, ft["k"][sl], ft["v"][sl], ft["alpha"][sl], beta(sl),
+                                          bf16_state=sdt == torch.bfloat16)
+        _, Oref = oracle.exact_steps(kind, S0, ft["k"][sl], ft["v"][sl], ft["alpha"][sl], beta(sl), ft["q"][sl])
+        tol = STATE_TOL if sdt == torch.float32 else BF16_STATE_TOL
+        assert state_err(to_logical(S), Sref) <= tol, n
+        assert state_err(P.reshape(B * H, dv, r).double().cpu().numpy(), Pref) <= tol, n
+        assert rel_l2(o.reshape(B * H, dv).cpu(), Oref[n - 1]) <= TIGHT_OUT, n
+
+
+@pytest.mark.parametrize("case", CASES, ids=[_ids(c) for c in CASES])
 def test_decode_step(case):
     import recurrent_state_read_b200 as rs
 
@@ -119,6 +150,45 @@ def test_decode_step(case):
                                  ft["alpha"][sl], None if ft["beta"] is None else ft["beta"][sl])
         err = rel_l2(o.reshape(B * H, dv).cpu(), ref)
         assert err <= TIGHT_OUT, (j, err)
+
+
+@pytest.mark.parametrize("case", CASES, ids=[_ids(c) for c in CASES])
+def test_replay_decode_step(case):
+    """ReplaySSM-style step j: the exact read of the window-start state through the buffered tokens
+    equals the oracle's per-step exact read S_j^T q_j; the state is not written."""
+    import recurrent_state_read_b200 as rs
+
+    kind, dk, dv, r, W, sdt, qdt = case
+    cfg, d, S0, U, R, tok = _setup(kind, dk, dv, r, W, sdt, qdt, seed=6)
+    B, H = d.B, d.H
+    ft = flat_tokens(tok)
+    dev = to_device(tok)
+    win = to_window(dev)
+    S = to_gpu_state(S0, B, H, sdt)
+    S_before = S.clone()
+    _, Oref = oracle.exact_steps(kind, S0, ft["k"], ft["v"], ft["alpha"], ft["beta"], ft["q"])
+    for j in sorted({1, max(1, W // 2), W}):
+        o = torch.full((B, H, dv), float("nan"), device="cuda")
+        rs.sketchssm_replay_decode_step(d, S, dev["q"][j - 1], win["k"], win["v"], win["alpha"], win["beta"], j, o)
+        torch.cuda.synchronize()
+        assert rel_l2(o.reshape(B * H, dv).cpu(), Oref[j - 1]) <= TIGHT_OUT, j
+    assert torch.equal(S, S_before)
+
+
+def test_update_window_without_sketch():
+    """P = NULL: the state update alone (the ReplaySSM-style window end), same state as with a refresh."""
+    import recurrent_state_read_b200 as rs
+
+    kind, dk, dv, r, W = "gdn", 128, 128, 8, 16
+    cfg, d, S0, U, R, tok = _setup(kind, dk, dv, r, W, torch.float32, torch.bfloat16, seed=7)
+    B, H = d.B, d.H
+    ft = flat_tokens(tok)
+    win = to_window(to_device(tok))
+    S = to_gpu_state(S0, B, H)
+    rs.sketchssm_update_window(d, S, None, None, win["k"], win["v"], win["alpha"], win["beta"], W)
+    torch.cuda.synchronize()
+    Sref, _ = oracle.exact_steps(kind, S0, ft["k"], ft["v"], ft["alpha"], ft["beta"])
+    assert state_err(to_logical(S), Sref) <= STATE_TOL
 
 
 @pytest.mark.parametrize("case", CASES, ids=[_ids(c) for c in CASES])

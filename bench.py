@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--stagger-share", default="2,2",
+                    help="CTAs per SM for the decode and update kernels of the staggered schedule")
     return ap.parse_args()
 
 
@@ -396,6 +398,29 @@ def run_ours(args):
     g_full = [capture(full_fn(tok)) for tok in toks]
     # the variant whose last step of each window is read exactly inside the window update
     g_x = [capture(lambda b=b: sketch_window(d, S, P, U, R, b, out, exact_last=True)) for b in bufs]
+    # the staggered schedule: sequence b's windows run with a phase of b mod W steps; at every step the
+    # sequences inside a window take a sketch step while those whose window ends are updated and read
+    # exactly, on a second stream (W steps per graph = every sequence through one whole window)
+    from recurrent_state_read_b200.decode import stagger_plan, staggered_step
+    plan = stagger_plan(cfg.B, cfg.W, dev)
+    share = tuple(int(x) for x in args.stagger_share.split(","))
+    side = torch.cuda.Stream(device=dev)
+    Sg, Pg = S.clone(), P.clone()
+
+    def stagger_cycle(b):
+        def fn():
+            for st in range(cfg.W):
+                fork = torch.cuda.Event()
+                fork.record(stream)
+                side.wait_event(fork)
+                staggered_step(d, Sg, Pg, U, R, b, b.q[st], plan[st], out[st], share,
+                               (stream.cuda_stream, side.cuda_stream))
+                join = torch.cuda.Event()
+                join.record(side)
+                stream.wait_event(join)
+        return fn
+
+    g_st = [capture(stagger_cycle(b)) for b in bufs]
     # the ReplaySSM-style baseline: W full-state reads of the window-start state + one update (no sketch)
     Sr = S0.clone()
     g_rdec = [capture(lambda b=b: [rs.sketchssm_replay_decode_step(d, Sr, b.q[j - 1], b.k, b.v, b.alpha, b.beta,
@@ -471,6 +496,20 @@ def run_ours(args):
     barrier()
     clocks.mark(False)
     t_x = max_over_ranks(xe0.elapsed_time(xe1) / 1e3)
+
+    # --- staggered schedule
+    for i in range(args.warmup):
+        g_st[i % NWIN].replay()
+    barrier()
+    se0, se1 = ev(), ev()
+    clocks.mark(True)
+    se0.record(stream)
+    for i in range(args.steps):
+        g_st[i % NWIN].replay()
+    se1.record(stream)
+    barrier()
+    clocks.mark(False)
+    t_st = max_over_ranks(se0.elapsed_time(se1) / 1e3)
 
     # --- ReplaySSM-style baseline
     for i in range(args.warmup):
@@ -564,6 +603,14 @@ def run_ours(args):
             "replay_step_GBps": bm["replay_avg"] / (1e3 * t_rdec / (args.steps * cfg.W)) / 1e6,
             "algorithmic_bytes_per_token_step": bm["replay_step"] / tok_per_step,
             "sketch_speedup": value / whole_job_rate(args.steps * tok_per_step, world, t_r)},
+        "staggered": {
+            "value": whole_job_rate(args.steps * tok_per_step, world, t_st), "unit": UNIT,
+            "ms_per_step": 1e3 * t_st / args.steps,
+            "schedule": f"sequence b's windows offset by b mod {cfg.W} steps; per decode step the sequences "
+                        f"inside a window take a sketch step (per-sequence step index) while about B/W "
+                        f"sequences end their window: update + exact read, concurrently on a second stream; "
+                        f"one step of this key = {cfg.W} decode steps = every sequence through one window",
+            "ctas_per_sm": {"decode": share[0], "update": share[1]}},
         "exact_last_step": {
             "value": whole_job_rate(args.steps * tok_per_step, world, t_x), "unit": UNIT,
             "ms_per_step": 1e3 * t_x / args.steps,
@@ -587,7 +634,7 @@ def run_ours(args):
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del g_dec, g_upd, g_full, g_x, g_rdec, g_rupd
+    del g_dec, g_upd, g_full, g_x, g_rdec, g_rupd, g_st
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

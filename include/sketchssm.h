@@ -154,6 +154,47 @@ int sketchssm_decode_step(const sketchssm_dims *dims, const float *P, const floa
                           const float *beta, int j, float *o, void *stream);
 
 /*
+ * sketchssm_decode_step_seq -- sketchssm_decode_step with a step index per
+ * sequence.  In serving, sequences reach the ends of their windows at different
+ * decode steps (they start at different times); j_seq[b] is sequence b's step
+ * within its own window, 1..W, or 0 for a sequence that takes no sketch step now
+ * (for instance, its window ends at this step and sketchssm_update_window_seqs
+ * reads it exactly).  Heads of a sequence with j_seq[b] == 0 keep their o.
+ *   j_seq  in device [B] int32 (4-byte aligned).  A value outside 0..W is counted
+ *          by sketchssm_device_error_count and that sequence is skipped.
+ *   sm_share  0: use the whole GPU; n > 0: at most n CTAs per SM, leaving room for a
+ *          kernel that runs at the same time on another stream (the window updates
+ *          of other sequences).
+ * Other arguments as sketchssm_decode_step.
+ * Errors: ERR_NULL, ERR_DIMS, ERR_DTYPE, ERR_RANGE (sm_share < 0), ERR_ALIGN, ERR_CUDA.
+ */
+int sketchssm_decode_step_seq(const sketchssm_dims *dims, const float *P, const float *R, const void *q,
+                              const void *k, const void *v, const float *alpha, const float *beta,
+                              const int32_t *j_seq, int sm_share, float *o, void *stream);
+
+/*
+ * sketchssm_update_window_seqs -- the window update (sketchssm_update_window, or
+ * with q and o sketchssm_update_window_read) for the n_seqs sequences listed in
+ * seqs only: every head of each listed sequence; the other sequences' state,
+ * sketch and output are not touched.  Sequences whose windows end at this step
+ * are updated while the others take sketch steps (sketchssm_decode_step_seq on
+ * another stream, both with sm_share > 0, so that the two kernels share the GPU).
+ *   seqs   in device [n_seqs] int32 sequence indices (4-byte aligned), 0 <= n_seqs <= B;
+ *          an index outside 0..B-1 is counted by sketchssm_device_error_count and
+ *          skipped.
+ *   q, o   both NULL (no read) or both given (the exact read, as
+ *          sketchssm_update_window_read).
+ *   P, U   as sketchssm_update_window (P NULL: no sketch refresh).
+ *   sm_share  as sketchssm_decode_step_seq.
+ * Errors: ERR_NULL, ERR_DIMS, ERR_DTYPE, ERR_RANGE (n_tokens, n_seqs, sm_share), ERR_ALIGN,
+ * ERR_CUDA.
+ */
+int sketchssm_update_window_seqs(const sketchssm_dims *dims, void *S, float *P, const float *U,
+                                 const void *k, const void *v, const float *alpha, const float *beta,
+                                 int n_tokens, const int32_t *seqs, int n_seqs, const void *q, float *o,
+                                 int sm_share, void *stream);
+
+/*
  * sketchssm_fullread_decode -- the baseline: one decode step with a full-state
  * read, as a standard serving engine does it (SketchSSM abstract, "standard
  * vLLM baseline"; digest bullet "Background": the full recurrent state is read
@@ -193,6 +234,9 @@ int sketchssm_replay_decode_step(const sketchssm_dims *dims, const void *S, cons
  * fixed number of attempts, count the give-up in a device-side counter and
  * return without writing that head's results (the window update also stops
  * the rest of its CTA's heads, leaving their state and sketch as they were).
+ * Per-sequence step indices and sequence indices out of range (read on the
+ * device by sketchssm_decode_step_seq and sketchssm_update_window_seqs) are
+ * counted the same way.
  * This call synchronises the current device and returns the sum of both counts
  * (0 in normal operation; a negative sketchssm_status if a CUDA call fails);
  * reset != 0 clears them.

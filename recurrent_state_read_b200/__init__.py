@@ -33,6 +33,8 @@ EXPORTS = (
     "sketchssm_update_window",
     "sketchssm_update_window_read",
     "sketchssm_decode_step",
+    "sketchssm_decode_step_seq",
+    "sketchssm_update_window_seqs",
     "sketchssm_fullread_decode",
     "sketchssm_replay_decode_step",
     "sketchssm_calibrate_workspace_bytes",
@@ -77,6 +79,8 @@ def library() -> ctypes.CDLL:
         lib.sketchssm_update_window.argtypes = [D, P, P, P, P, P, P, P, i, P]
         lib.sketchssm_update_window_read.argtypes = [D, P, P, P, P, P, P, P, i, P, P, P]
         lib.sketchssm_decode_step.argtypes = [D, P, P, P, P, P, P, P, i, P, P]
+        lib.sketchssm_decode_step_seq.argtypes = [D, P, P, P, P, P, P, P, P, i, P, P]
+        lib.sketchssm_update_window_seqs.argtypes = [D, P, P, P, P, P, P, P, i, P, i, P, P, i, P]
         lib.sketchssm_fullread_decode.argtypes = [D, P, P, P, P, P, P, P, P]
         lib.sketchssm_replay_decode_step.argtypes = [D, P, P, P, P, P, P, i, P, P]
         lib.sketchssm_calibrate_workspace_bytes.argtypes = [D, i, i]
@@ -87,7 +91,7 @@ def library() -> ctypes.CDLL:
         lib.sketchssm_device_error_count.argtypes = [i]
         lib.sketchssm_device_error_count.restype = i
         for f in ("sketchssm_update_window", "sketchssm_update_window_read", "sketchssm_decode_step",
-                  "sketchssm_replay_decode_step", "sketchssm_fullread_decode",
+                  "sketchssm_replay_decode_step", "sketchssm_decode_step_seq", "sketchssm_update_window_seqs", "sketchssm_fullread_decode",
                   "sketchssm_calibrate_basis", "sketchssm_calibrate_basis_noalloc"):
             getattr(lib, f).restype = i
         _lib = lib
@@ -177,6 +181,45 @@ def sketchssm_decode_step(d: sketchssm_dims, P, R, q, k, v, alpha, beta, j: int,
         ctypes.byref(d), _ptr(P, "P", NH * d.dv * d.r, torch.float32),
         _ptr(R, "R", d.H * d.r * d.dk, torch.float32), _ptr(q, "q", NH * d.dk, _dt(d.qkv_dtype)),
         *toks, int(j), _ptr(o, "o", NH * d.dv, torch.float32), ctypes.c_void_p(_stream(stream))))
+
+
+def _i32(t, name, numel):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.int32 or not t.is_contiguous():
+        raise TypeError(f"{name}: expected a contiguous int32 CUDA tensor")
+    if t.numel() < numel:
+        raise ValueError(f"{name}: needs at least {numel} elements, has {t.numel()}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def sketchssm_decode_step_seq(d: sketchssm_dims, P, R, q, k, v, alpha, beta, j_seq, o, sm_share: int = 0,
+                              stream=None):
+    """Decode step with a step index per sequence (j_seq: int32 [B] on the device, 1..W, or 0 for no
+    step); sm_share > 0 caps the CTAs per SM so that a concurrent kernel fits."""
+    NH = d.B * d.H
+    toks = _token_ptrs(d, d.W, k, v, alpha, beta)
+    _check("sketchssm_decode_step_seq", library().sketchssm_decode_step_seq(
+        ctypes.byref(d), _ptr(P, "P", NH * d.dv * d.r, torch.float32),
+        _ptr(R, "R", d.H * d.r * d.dk, torch.float32), _ptr(q, "q", NH * d.dk, _dt(d.qkv_dtype)),
+        *toks, _i32(j_seq, "j_seq", d.B), int(sm_share), _ptr(o, "o", NH * d.dv, torch.float32),
+        ctypes.c_void_p(_stream(stream))))
+
+
+def sketchssm_update_window_seqs(d: sketchssm_dims, S, P, U, k, v, alpha, beta, n_tokens: int, seqs,
+                                 q=None, o=None, sm_share: int = 0, stream=None):
+    """The window update (and with q, o the exact read) for the sequences listed in seqs (int32 on the
+    device) only."""
+    NH = d.B * d.H
+    n_seqs = int(seqs.numel())
+    toks = _token_ptrs(d, d.W, k, v, alpha, beta) if n_tokens > 0 else (None,) * 4
+    _check("sketchssm_update_window_seqs", library().sketchssm_update_window_seqs(
+        ctypes.byref(d), _ptr(S, "S", NH * d.dv * d.dk, _dt(d.state_dtype)),
+        None if P is None else _ptr(P, "P", NH * d.dv * d.r, torch.float32),
+        None if U is None else _ptr(U, "U", d.H * d.dk * d.r, torch.float32), *toks, int(n_tokens),
+        _i32(seqs, "seqs", n_seqs), n_seqs, None if q is None else _ptr(q, "q", NH * d.dk, _dt(d.qkv_dtype)),
+        None if o is None else _ptr(o, "o", NH * d.dv, torch.float32), int(sm_share),
+        ctypes.c_void_p(_stream(stream))))
 
 
 def sketchssm_replay_decode_step(d: sketchssm_dims, S, q, k, v, alpha, beta, j: int, o, stream=None):

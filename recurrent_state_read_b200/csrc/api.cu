@@ -66,8 +66,8 @@ int sketchssm_update_window(const sketchssm_dims *d, void *S, float *P, const fl
     if (n_tokens < 0 || n_tokens > d->W) return SKSSM_ERR_RANGE;
     if (n_tokens > 0 && (rc = check_tokens(d, k, v, alpha, beta))) return rc;
     if (!aligned(S, 16) || !aligned(P, 16) || !aligned(U, 16)) return SKSSM_ERR_ALIGN;
-    return launch_update_window(*d, S, P, P ? U : nullptr, k, v, alpha, beta, n_tokens, nullptr, nullptr,
-                                (cudaStream_t)stream);
+    return launch_update_window(*d, S, P, P ? U : nullptr, k, v, alpha, beta, n_tokens, nullptr, nullptr, nullptr,
+                                0, 0, (cudaStream_t)stream);
 }
 
 int sketchssm_update_window_read(const sketchssm_dims *d, void *S, float *P, const float *U, const void *k,
@@ -80,7 +80,7 @@ int sketchssm_update_window_read(const sketchssm_dims *d, void *S, float *P, con
     if (n_tokens > 0 && (rc = check_tokens(d, k, v, alpha, beta))) return rc;
     if (!aligned(S, 16) || !aligned(P, 16) || !aligned(U, 16) || !aligned(q, 16) || !aligned(o, 16))
         return SKSSM_ERR_ALIGN;
-    return launch_update_window(*d, S, P, U, k, v, alpha, beta, n_tokens, q, o, (cudaStream_t)stream);
+    return launch_update_window(*d, S, P, U, k, v, alpha, beta, n_tokens, q, o, nullptr, 0, 0, (cudaStream_t)stream);
 }
 
 int sketchssm_decode_step(const sketchssm_dims *d, const float *P, const float *R, const void *q,
@@ -92,7 +92,7 @@ int sketchssm_decode_step(const sketchssm_dims *d, const float *P, const float *
     if (j < 1 || j > d->W) return SKSSM_ERR_RANGE;
     if ((rc = check_tokens(d, k, v, alpha, beta))) return rc;
     if (!aligned(P, 16) || !aligned(R, 16) || !aligned(q, 16) || !aligned(o, 16)) return SKSSM_ERR_ALIGN;
-    return launch_decode_step(*d, P, R, q, k, v, alpha, beta, j, o, (cudaStream_t)stream);
+    return launch_decode_step(*d, P, R, q, k, v, alpha, beta, j, nullptr, 0, o, (cudaStream_t)stream);
 }
 
 int sketchssm_fullread_decode(const sketchssm_dims *d, void *S, const void *q, const void *k,
@@ -104,6 +104,35 @@ int sketchssm_fullread_decode(const sketchssm_dims *d, void *S, const void *q, c
     if ((rc = check_tokens(d, k, v, alpha, beta))) return rc;
     if (!aligned(S, 16) || !aligned(q, 16) || !aligned(o, 16)) return SKSSM_ERR_ALIGN;
     return launch_fullread(*d, S, q, k, v, alpha, beta, o, (cudaStream_t)stream);
+}
+
+int sketchssm_decode_step_seq(const sketchssm_dims *d, const float *P, const float *R, const void *q, const void *k,
+                              const void *v, const float *alpha, const float *beta, const int32_t *j_seq,
+                              int sm_share, float *o, void *stream) {
+    int rc = check_dims(d);
+    if (rc) return rc;
+    if (!P || !R || !q || !o || !j_seq) return SKSSM_ERR_NULL;
+    if (sm_share < 0) return SKSSM_ERR_RANGE;
+    if ((rc = check_tokens(d, k, v, alpha, beta))) return rc;
+    if (!aligned(P, 16) || !aligned(R, 16) || !aligned(q, 16) || !aligned(o, 16) || !aligned(j_seq, 4))
+        return SKSSM_ERR_ALIGN;
+    return launch_decode_step(*d, P, R, q, k, v, alpha, beta, d->W, j_seq, sm_share, o, (cudaStream_t)stream);
+}
+
+int sketchssm_update_window_seqs(const sketchssm_dims *d, void *S, float *P, const float *U, const void *k,
+                                 const void *v, const float *alpha, const float *beta, int n_tokens,
+                                 const int32_t *seqs, int n_seqs, const void *q, float *o, int sm_share,
+                                 void *stream) {
+    int rc = check_dims(d);
+    if (rc) return rc;
+    if (!S || (P && !U) || !seqs || (!q != !o)) return SKSSM_ERR_NULL;
+    if (n_tokens < 0 || n_tokens > d->W || n_seqs < 0 || n_seqs > d->B || sm_share < 0) return SKSSM_ERR_RANGE;
+    if (n_tokens > 0 && (rc = check_tokens(d, k, v, alpha, beta))) return rc;
+    if (!aligned(S, 16) || !aligned(P, 16) || !aligned(U, 16) || !aligned(q, 16) || !aligned(o, 16) ||
+        !aligned(seqs, 4))
+        return SKSSM_ERR_ALIGN;
+    return launch_update_window(*d, S, P, P ? U : nullptr, k, v, alpha, beta, n_tokens, q, o, seqs, n_seqs, sm_share,
+                                (cudaStream_t)stream);
 }
 
 int sketchssm_replay_decode_step(const sketchssm_dims *d, const void *S, const void *q, const void *k, const void *v,

@@ -65,7 +65,8 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
 decode_step_kernel(const float *__restrict__ P, const float *__restrict__ R, const QT *__restrict__ qv,
                    const QT *__restrict__ kbuf, const QT *__restrict__ vbuf,
                    const float *__restrict__ abuf, const float *__restrict__ bbuf,
-                   float *__restrict__ o, int B, int H, int r, int j, int W, int jc) {
+                   float *__restrict__ o, int B, int H, int r, int j, int W, int jc,
+                   const int *__restrict__ jv) {
     using SL = DecSlots<KIND, DK, DV, QT>;
     constexpr int KPL = DK / 32, VPL = DV / 32;  // channels of the carried query / output per lane
     extern __shared__ __align__(16) char smem[];
@@ -75,6 +76,14 @@ decode_step_kernel(const float *__restrict__ P, const float *__restrict__ R, con
     if (oi >= NH) return;  // the whole warp
     const int h = oi / B;
     const int head = (oi % B) * H + h;
+    if (jv != nullptr) {  // the step of this head's sequence within its own window
+        j = jv[oi % B];
+        if (j < 0 || j > W) {
+            if (lane == 0) atomicAdd(&g_device_error, 1u);
+            return;
+        }
+        if (j == 0) return;  // the sequence takes no sketch step now
+    }
     char *wb = smem + (size_t)warp * SL::bytes(jc);
     uint64_t *bar = reinterpret_cast<uint64_t *>(wb);
     char *ks = wb + 16, *vs = ks + jc * SL::KB, *as = vs + jc * SL::VB;
@@ -205,12 +214,12 @@ struct DecStage {
     __host__ __device__ static int bytes(int j) { return QB + tokens(j); }
 };
 
-template <int KIND, int DK, int DV, typename QT>
+template <int KIND, int DK, int DV, typename QT, bool JV>
 __global__ void __launch_bounds__(DEC_WARPS * 32)
 decode_step_persistent(const float *__restrict__ P, const float *__restrict__ R, const QT *__restrict__ qv,
                        const QT *__restrict__ kbuf, const QT *__restrict__ vbuf,
                        const float *__restrict__ abuf, const float *__restrict__ bbuf,
-                       float *__restrict__ o, int B, int H, int r, int j, int W) {
+                       float *__restrict__ o, int B, int H, int r, int j, int W, const int *__restrict__ jv) {
     using SL = DecSlots<KIND, DK, DV, QT>;
     using STG = DecStage<KIND, DK, DV, QT>;
     constexpr int KPL = DK / 32, VPL = DV / 32;
@@ -227,21 +236,35 @@ decode_step_persistent(const float *__restrict__ P, const float *__restrict__ R,
     const int i1 = min(NH, i0 + per);
     if (i0 >= i1) return;  // the whole warp; the kernel has no CTA-wide barrier
 
-    // every lane starts its share of the 16-byte copies of one head into stage s (one commit group)
-    auto issue = [&](int head, int s) {
+    // every lane starts its share of the 16-byte copies of one head's jh tokens into stage s (one
+    // commit group, empty when the head takes no step); stages are sized for j tokens, j >= jh
+    auto issue = [&](int head, int jh, int s) {
         char *sb = stage0 + s * sbytes;
         char *qs = sb, *ks = qs + STG::QB, *vs = ks + j * SL::KB, *as = vs + j * SL::VB;
-        copy16(qs, qv + (size_t)head * DK, STG::QB, lane);
-        copy16(ks, kbuf + (size_t)head * W * DK, j * SL::KB, lane);
-        copy16(vs, vbuf + (size_t)head * W * DV, j * SL::VB, lane);
-        if (KIND == KDA) copy16(as, abuf + (size_t)head * W * DK, j * SL::AB, lane);
+        if (jh > 0) {
+            copy16(qs, qv + (size_t)head * DK, STG::QB, lane);
+            copy16(ks, kbuf + (size_t)head * W * DK, jh * SL::KB, lane);
+            copy16(vs, vbuf + (size_t)head * W * DV, jh * SL::VB, lane);
+            if (KIND == KDA) copy16(as, abuf + (size_t)head * W * DK, jh * SL::AB, lane);
+        }
         asm volatile("cp.async.commit_group;\n" ::: "memory");
+    };
+    // the step of sequence b within its own window (every head of the call when jv is NULL); an index
+    // outside 0..j is counted as a device error and the head is skipped
+    auto step_of = [&](int b) -> int {
+        if constexpr (!JV) return j;
+        const int jh = jv[b];
+        if (jh < 0 || jh > j) {
+            if (lane == 0) atomicAdd(&g_device_error, 1u);
+            return 0;
+        }
+        return jh;
     };
     // every lane: the per-token scalars of one head (token t in lane t, j <= 32) and the first
     // DEC_RPRE sketch columns of the lane's value channels, into registers
-    auto scalars = [&](int head, float &al, float &bl, float (&pp)[VPL][DEC_RPRE]) {
-        al = (KIND != KDA && lane < j) ? abuf[(size_t)head * W + lane] : 1.f;
-        bl = (KIND != MAMBA2 && lane < j) ? bbuf[(size_t)head * W + lane] : 1.f;
+    auto scalars = [&](int head, int jh, float &al, float &bl, float (&pp)[VPL][DEC_RPRE]) {
+        al = (KIND != KDA && lane < jh) ? abuf[(size_t)head * W + lane] : 1.f;
+        bl = (KIND != MAMBA2 && lane < jh) ? bbuf[(size_t)head * W + lane] : 1.f;
         const float *Ph = P + (size_t)head * DV * r;
 #pragma unroll
         for (int e = 0; e < VPL; ++e) {
@@ -260,9 +283,11 @@ decode_step_persistent(const float *__restrict__ P, const float *__restrict__ R,
     int nh = i0 / B, nb = i0 - nh * B;  // the next head to issue
     int ch = nh, cb = nb;               // the head being computed
     float a_c, b_c, a_n = 1.f, b_n = 1.f, pp_c[VPL][DEC_RPRE], pp_n[VPL][DEC_RPRE];
-    issue(nb * H + nh, 0);
-    scalars(nb * H + nh, a_c, b_c, pp_c);
+    int j_c = step_of(nb);
+    issue(nb * H + nh, JV ? j_c : j, 0);
+    scalars(nb * H + nh, JV ? j_c : j, a_c, b_c, pp_c);
     if (++nb == B) { nb = 0; ++nh; }
+    int j_n = JV && i0 + 1 < i1 ? step_of(nb) : 0;  // the step of the next head, one head ahead of its copies
 
     int h_rows = -1;
     float rr[DEC_RPRE][KPL];
@@ -270,10 +295,12 @@ decode_step_persistent(const float *__restrict__ P, const float *__restrict__ R,
         const int s = it & 1;
         const int head = cb * H + ch;
         const bool more = i + 1 < i1;
+        int j_nn = 0;
         if (more) {
-            issue(nb * H + nh, s ^ 1);
-            scalars(nb * H + nh, a_n, b_n, pp_n);
+            issue(nb * H + nh, JV ? j_n : j, s ^ 1);
+            scalars(nb * H + nh, JV ? j_n : j, a_n, b_n, pp_n);
             if (++nb == B) { nb = 0; ++nh; }
+            if (JV && i + 2 < i1) j_nn = step_of(nb);
         }
         const float *Rh = R + (size_t)ch * r * DK;
         if (ch != h_rows) {  // warp-uniform
@@ -295,59 +322,63 @@ decode_step_persistent(const float *__restrict__ P, const float *__restrict__ R,
         const char *sb = stage0 + s * sbytes;
         const char *qs = sb, *ks = qs + STG::QB, *vs = ks + j * SL::KB, *as = vs + j * SL::VB;
 
-        float acc[VPL];
-        float w[KPL], ob[VPL];
-        load_n<KPL>(reinterpret_cast<const QT *>(qs) + lane * KPL, w);
+        if (!JV || j_c > 0) {  // warp-uniform
+            float acc[VPL];
+            float w[KPL], ob[VPL];
+            load_n<KPL>(reinterpret_cast<const QT *>(qs) + lane * KPL, w);
 #pragma unroll
-        for (int e = 0; e < VPL; ++e) ob[e] = 0.f;
-        float gsc = 1.f;
-        backward_chunk<KIND, DK, DV, QT>(ks, vs, as, j, a_c, b_c, w, ob, gsc, lane);
-        if (KIND != KDA) {
+            for (int e = 0; e < VPL; ++e) ob[e] = 0.f;
+            float gsc = 1.f;
+            backward_chunk<KIND, DK, DV, QT>(ks, vs, as, JV ? j_c : j, a_c, b_c, w, ob, gsc, lane);
+            if (KIND != KDA) {
 #pragma unroll
-            for (int e = 0; e < KPL; ++e) w[e] *= gsc;
-        }
+                for (int e = 0; e < KPL; ++e) w[e] *= gsc;
+            }
 
-        // c = R q~ (eight rows per warp all-reduce; rows past the first eight from L1/L2),
-        // o = P c + o_buf (the first eight sketch columns from registers, the rest from L1/L2)
-        const float *Ph = P + (size_t)head * DV * r;
+            // c = R q~ (eight rows per warp all-reduce; rows past the first eight from L1/L2),
+            // o = P c + o_buf (the first eight sketch columns from registers, the rest from L1/L2)
+            const float *Ph = P + (size_t)head * DV * r;
 #pragma unroll
-        for (int e = 0; e < VPL; ++e) acc[e] = ob[e];
+            for (int e = 0; e < VPL; ++e) acc[e] = ob[e];
 #pragma unroll 1
-        for (int m0 = 0; m0 < r; m0 += DEC_RPRE) {
-            float c[DEC_RPRE];
+            for (int m0 = 0; m0 < r; m0 += DEC_RPRE) {
+                float c[DEC_RPRE];
 #pragma unroll
-            for (int mm = 0; mm < DEC_RPRE; ++mm) {
-                c[mm] = 0.f;
-                if (m0 == 0) {
+                for (int mm = 0; mm < DEC_RPRE; ++mm) {
+                    c[mm] = 0.f;
+                    if (m0 == 0) {
 #pragma unroll
-                    for (int e = 0; e < KPL; ++e) c[mm] = fmaf(rr[mm][e], w[e], c[mm]);
-                } else if (m0 + mm < r) {
-                    float rv[KPL];
-                    load_n<KPL>(Rh + (size_t)(m0 + mm) * DK + lane * KPL, rv);
+                        for (int e = 0; e < KPL; ++e) c[mm] = fmaf(rr[mm][e], w[e], c[mm]);
+                    } else if (m0 + mm < r) {
+                        float rv[KPL];
+                        load_n<KPL>(Rh + (size_t)(m0 + mm) * DK + lane * KPL, rv);
 #pragma unroll
-                    for (int e = 0; e < KPL; ++e) c[mm] = fmaf(rv[e], w[e], c[mm]);
+                        for (int e = 0; e < KPL; ++e) c[mm] = fmaf(rv[e], w[e], c[mm]);
+                    }
+                }
+                warp_allreduce8(c, lane);
+#pragma unroll
+                for (int mm = 0; mm < DEC_RPRE; ++mm) {
+                    if (m0 == 0) {
+#pragma unroll
+                        for (int e = 0; e < VPL; ++e) acc[e] = fmaf(pp_c[e][mm], c[mm], acc[e]);
+                    } else if (m0 + mm < r) {
+#pragma unroll
+                        for (int e = 0; e < VPL; ++e)
+                            acc[e] = fmaf(Ph[(size_t)(lane * VPL + e) * r + m0 + mm], c[mm], acc[e]);
+                    }
                 }
             }
-            warp_allreduce8(c, lane);
-#pragma unroll
-            for (int mm = 0; mm < DEC_RPRE; ++mm) {
-                if (m0 == 0) {
-#pragma unroll
-                    for (int e = 0; e < VPL; ++e) acc[e] = fmaf(pp_c[e][mm], c[mm], acc[e]);
-                } else if (m0 + mm < r) {
-#pragma unroll
-                    for (int e = 0; e < VPL; ++e)
-                        acc[e] = fmaf(Ph[(size_t)(lane * VPL + e) * r + m0 + mm], c[mm], acc[e]);
-                }
-            }
+            float *oh = o + (size_t)head * DV + lane * VPL;
+            if constexpr (VPL == 4) *reinterpret_cast<float4 *>(oh) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            else *reinterpret_cast<float2 *>(oh) = make_float2(acc[0], acc[1]);
         }
-        float *oh = o + (size_t)head * DV + lane * VPL;
-        if constexpr (VPL == 4) *reinterpret_cast<float4 *>(oh) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        else *reinterpret_cast<float2 *>(oh) = make_float2(acc[0], acc[1]);
 
         __syncwarp();  // every lane is done with this stage before it is refilled
         a_c = a_n;
         b_c = b_n;
+        j_c = j_n;
+        j_n = j_nn;
 #pragma unroll
         for (int e = 0; e < VPL; ++e)
 #pragma unroll
@@ -358,7 +389,8 @@ decode_step_persistent(const float *__restrict__ P, const float *__restrict__ R,
 
 int launch_decode_step(const sketchssm_dims &d, const float *P, const float *R, const void *q,
                        const void *k, const void *v, const float *alpha, const float *beta, int j,
-                       float *o, cudaStream_t stream) {
+                       const int *jv, int sm_share, float *o, cudaStream_t stream) {
+    if (jv != nullptr) j = d.W;  // per-sequence steps: size everything for the longest
     // the kernel does not touch the state: both state dtypes dispatch to the same instantiation
     return dispatch(d, [&](auto K, auto D, auto *, auto *qp) -> int {
         using QT = std::remove_pointer_t<decltype(qp)>;
@@ -371,25 +403,33 @@ int launch_decode_step(const sketchssm_dims &d, const float *P, const float *R, 
             if (j <= 32) {
                 const size_t psmem = (size_t)DEC_WARPS * 2 * DecStage<KIND, DK, DV, QT>::bytes(j);
                 if (psmem <= 227 * 1024) {
-                    auto pk = decode_step_persistent<KIND, DK, DV, QT>;
-                    static bool p_opted_in = false;
-                    if (!p_opted_in) {
-                        if (cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-                            cudaSuccess)
+                    // per-sequence steps are a separate instantiation: their checks cost the uniform
+                    // step a few percent (measured)
+                    auto persist = [&](auto JVc) -> int {
+                        auto pk = decode_step_persistent<KIND, DK, DV, QT, decltype(JVc)::value>;
+                        static bool p_opted_in = false;
+                        if (!p_opted_in) {
+                            if (cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+                                cudaSuccess)
+                                return SKSSM_ERR_CUDA;
+                            p_opted_in = true;
+                        }
+                        int sms = 0, per_sm = 0;
+                        if (sm_count(&sms) != SKSSM_OK ||
+                            blocks_per_sm(reinterpret_cast<const void *>(pk), DEC_WARPS * 32, psmem, &per_sm) !=
+                                SKSSM_OK)
                             return SKSSM_ERR_CUDA;
-                        p_opted_in = true;
-                    }
-                    int sms = 0, per_sm = 0;
-                    if (sm_count(&sms) != SKSSM_OK ||
-                        blocks_per_sm(reinterpret_cast<const void *>(pk), DEC_WARPS * 32, psmem, &per_sm) != SKSSM_OK)
-                        return SKSSM_ERR_CUDA;
-                    if (per_sm * DEC_WARPS >= DEC_PERSIST_MIN_WARPS) {
+                        if (sm_share > 0 && sm_share < per_sm) per_sm = sm_share;  // leave room for another kernel
+                        if (per_sm < 1 || (per_sm * DEC_WARPS < DEC_PERSIST_MIN_WARPS && sm_share == 0))
+                            return 1;  // not taken: the one-head-per-warp kernel below
                         const int pgrid = grid < sms * per_sm ? grid : sms * per_sm;
                         pk<<<pgrid, DEC_WARPS * 32, psmem, stream>>>(
                             P, R, static_cast<const QT *>(q), static_cast<const QT *>(k), static_cast<const QT *>(v),
-                            alpha, beta, o, d.B, d.H, d.r, j, d.W);
+                            alpha, beta, o, d.B, d.H, d.r, j, d.W, jv);
                         return launch_status();
-                    }
+                    };
+                    const int rc = jv != nullptr ? persist(std::true_type()) : persist(std::false_type());
+                    if (rc != 1) return rc;
                 }
             }
             // tokens per bulk round trip (<= 32: one per lane); KDA rows are twice as wide, and fewer
@@ -407,7 +447,7 @@ int launch_decode_step(const sketchssm_dims &d, const float *P, const float *R, 
             }
             kern<<<grid, DEC_WARPS * 32, smem, stream>>>(P, R, static_cast<const QT *>(q),
                                                          static_cast<const QT *>(k), static_cast<const QT *>(v),
-                                                         alpha, beta, o, d.B, d.H, d.r, j, d.W, jc);
+                                                         alpha, beta, o, d.B, d.H, d.r, j, d.W, jc, jv);
             return launch_status();
         };
         if (d.dv == 64) return go(std::integral_constant<int, 64>());

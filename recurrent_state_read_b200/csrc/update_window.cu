@@ -28,6 +28,9 @@
 namespace skssm {
 
 constexpr int UPD_NC = 8;  // value columns per lane (state_tile.cuh)
+
+// bounded waits that gave up, and sequence indices out of range, in either update kernel
+__device__ unsigned g_update_wait_giveups;
 constexpr int PER_NC = 4;      // the same for the persistent kernel
 constexpr int PER_STAGES = 1;  // shared-memory stages per persistent CTA: with one stage more CTAs fit on an
                                // SM, which hides the copies better than a deeper pipeline per CTA (measured)
@@ -81,7 +84,7 @@ __device__ __forceinline__ void stage_rows(const T *__restrict__ src, size_t row
 // Steps shared by both window-update kernels, for one head whose state is in
 // registers: apply the n staged tokens in order, scale, round to the storage
 // type, store the state once, and refresh the sketch from the same registers.
-template <int KIND, int DK, typename ST, int NC>
+template <int KIND, int DK, typename ST, int NC, bool READ>
 __device__ __forceinline__ void apply_store_refresh(float (&s)[NC][DK / 8], const float *sk, const float *su,
                                                     const float *sv, const float *sg, const float *sut,
                                                     const float *ss2, const float *sq, ST *__restrict__ S,
@@ -138,7 +141,7 @@ __device__ __forceinline__ void apply_store_refresh(float (&s)[NC][DK / 8], cons
     }
     // the exact read of the window's last step, o = S^T q, from the updated fp32 state (the
     // full-read step reads before storage rounding too)
-    if (sq != nullptr) {
+    if constexpr (READ) {
         float qv[EPL];
         lane_channels_smem<DK, ST>(sq, l, qv);
         float d[NC];
@@ -192,20 +195,27 @@ __device__ __forceinline__ void apply_store_refresh(float (&s)[NC][DK / 8], cons
     }
 }
 
-template <int KIND, int DK, typename ST, typename QT, int NC>
+template <int KIND, int DK, typename ST, typename QT, int NC, bool READ, bool SEQS>
 __global__ void __launch_bounds__(256)
 update_window_kernel(ST *__restrict__ S, float *__restrict__ P, const float *__restrict__ U,
                      const QT *__restrict__ kbuf, const QT *__restrict__ vbuf,
                      const float *__restrict__ abuf, const float *__restrict__ bbuf,
                      const QT *__restrict__ qv, float *__restrict__ o, int B, int H,
-                     int dv, int r, int n, int W) {
+                     int dv, int r, int n, int W, const int *__restrict__ seqs, int n_seqs) {
     using TL = TileLayout<DK, ST>;
     constexpr int EPL = TL::EPL;
     extern __shared__ __align__(16) float smem[];
 
-    // heads in (h, b) order: neighbouring CTAs share their basis rows in L2
-    const int h = blockIdx.x / B;
-    const int head = (blockIdx.x % B) * H + h;
+    // heads in (h, b) order: neighbouring CTAs share their basis rows in L2; the call's sequences
+    // are all B or the n_seqs listed in seqs (an index outside 0..B-1 is counted and skipped)
+    const int NB = SEQS ? n_seqs : B;
+    const int h = blockIdx.x / NB;
+    const int b = SEQS ? seqs[blockIdx.x % NB] : blockIdx.x % NB;
+    if (SEQS && (b < 0 || b >= B)) {
+        if (threadIdx.x == 0) atomicAdd(&g_update_wait_giveups, 1u);
+        return;  // the whole CTA
+    }
+    const int head = b * H + h;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int l = lane & 7, g = lane >> 3;
     const int c0 = warp * 4 * NC + g * NC;
@@ -231,7 +241,7 @@ update_window_kernel(ST *__restrict__ S, float *__restrict__ P, const float *__r
         const float4 *src = reinterpret_cast<const float4 *>(U + (size_t)h * r * DK);
         for (int i = tid; i < r * DK / 4; i += nthr) reinterpret_cast<float4 *>(sut)[i] = src[i];
     }
-    if (qv != nullptr)
+    if constexpr (READ)
         for (int i = tid; i < DK; i += nthr) sq[i] = ld1(qv + (size_t)head * DK + i);
     if (KIND != KDA) {
         if (warp == 0) {
@@ -274,7 +284,7 @@ update_window_kernel(ST *__restrict__ S, float *__restrict__ P, const float *__r
     }
     __syncthreads();
 
-    apply_store_refresh<KIND, DK, ST, NC>(s, sk, su, sv, sg, sut, ss2, qv ? sq : nullptr, S, P, o, head, dv, r, n,
+    apply_store_refresh<KIND, DK, ST, NC, READ>(s, sk, su, sv, sg, sut, ss2, sq, S, P, o, head, dv, r, n,
                                           c0, l, lane);
 }
 
@@ -289,7 +299,6 @@ update_window_kernel(ST *__restrict__ S, float *__restrict__ P, const float *__r
 // (sketchssm_device_error_count) and the CTA returns.
 // ---------------------------------------------------------------------------
 
-__device__ unsigned g_update_wait_giveups;
 constexpr unsigned UPD_WAIT_TRIES = 1u << 22;
 
 __device__ __forceinline__ unsigned upd_smem(const void *p) { return (unsigned)__cvta_generic_to_shared(p); }
@@ -324,14 +333,14 @@ struct PerLayout {
 };
 
 __host__ __device__ inline PerLayout per_layout(int kind, int DK, int dv, int r, int n, int sbytes, int qbytes,
-                                                int ns) {
+                                                int ns, bool read) {
     PerLayout L;
     int t = 0;
     L.st = t; t += up16(dv * DK * sbytes);
     L.kr = t; t += up16(n * DK * qbytes);
     L.vr = t; t += up16(n * dv * qbytes);
     L.ar = t; t += kind == KDA ? up16(n * DK * 4) : 0;
-    L.qr = t; t += up16(DK * qbytes);
+    L.qr = t; t += read ? up16(DK * qbytes) : 0;
     L.stage_bytes = t;
     int off = 16 * 2;  // two mbarriers, 16 bytes apart
     L.stages = off; off += ns * t;
@@ -341,24 +350,27 @@ __host__ __device__ inline PerLayout per_layout(int kind, int DK, int dv, int r,
     L.sg = off; off += up16(DK * 4);
     L.sut = off; off += up16(r * DK * 4);
     L.ss2 = off; off += up16(n * 4);
-    L.sq = off; off += up16(DK * 4);
+    L.sq = off; off += read ? up16(DK * 4) : 0;
     L.total = off;
     return L;
 }
 
-template <int KIND, int DK, typename ST, typename QT, int NC>
+template <int KIND, int DK, typename ST, typename QT, int NC, bool READ, bool SEQS>
 __global__ void __launch_bounds__(256)
 update_window_persistent(ST *__restrict__ S, float *__restrict__ P, const float *__restrict__ U,
                          const QT *__restrict__ kbuf, const QT *__restrict__ vbuf,
                          const float *__restrict__ abuf, const float *__restrict__ bbuf,
                          const QT *__restrict__ qv, float *__restrict__ o, int B, int H, int dv, int r, int n, int W,
-                         int ns) {
+                         int ns, const int *__restrict__ seqs, int n_seqs) {
     using TL = TileLayout<DK, ST>;
     constexpr int EPL = TL::EPL;
     extern __shared__ __align__(128) float psm_f[];
     char *smem = reinterpret_cast<char *>(psm_f);
-    const PerLayout L = per_layout(KIND, DK, dv, r, n, sizeof(ST), sizeof(QT), ns);
-    const int NH = B * H;
+    const PerLayout L = per_layout(KIND, DK, dv, r, n, sizeof(ST), sizeof(QT), ns, READ);
+    // the call's sequences: all B, or the n_seqs listed in seqs (an index outside 0..B-1 is counted
+    // as a device error and its heads are skipped); work item w = (h, i) in (h, i) order
+    const int NB = SEQS ? n_seqs : B;
+    const int NH = NB * H;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int l = lane & 7, g = lane >> 3;
     const int c0 = warp * 4 * NC + g * NC;
@@ -367,7 +379,11 @@ update_window_persistent(ST *__restrict__ S, float *__restrict__ P, const float 
     const int per = (NH + gridDim.x - 1) / gridDim.x;
     const int w_begin = blockIdx.x * per;
     const int w_end = min(NH, w_begin + per);
-    auto head_of = [&](int w) { return (w % B) * H + w / B; };
+    auto head_of = [&](int w) -> int {
+        if constexpr (!SEQS) return (w % B) * H + w / B;
+        const int b = seqs[w % NB];
+        return (b >= 0 && b < B) ? b * H + w / NB : -1;
+    };
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
     float *sk = reinterpret_cast<float *>(smem + L.sk);
@@ -380,18 +396,23 @@ update_window_persistent(ST *__restrict__ S, float *__restrict__ P, const float 
     const int state_bytes = dv * DK * (int)sizeof(ST);
     const int kbytes = n * DK * (int)sizeof(QT), vbytes = n * dv * (int)sizeof(QT);
     const int abytes = KIND == KDA ? n * DK * 4 : 0;
-    const int qbytes = qv != nullptr ? DK * (int)sizeof(QT) : 0;
+    const int qbytes = READ ? DK * (int)sizeof(QT) : 0;
 
     auto issue = [&](int w, int stage) {  // one thread
         char *sb = smem + L.stages + stage * L.stage_bytes;
         const int head = head_of(w);
         uint64_t *bar = bars + 2 * stage;
+        if (SEQS && head < 0) {  // nothing to copy: complete the stage's phase at once
+            atomicAdd(&g_update_wait_giveups, 1u);
+            asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(upd_smem(bar)) : "memory");
+            return;
+        }
         asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(upd_smem(bar)),
                      "r"(state_bytes + kbytes + vbytes + abytes + qbytes)
                      : "memory");
         upd_bulk(sb + L.st, S + (size_t)head * dv * DK, state_bytes, bar);
-        if (qbytes) upd_bulk(sb + L.qr, qv + (size_t)head * DK, qbytes, bar);
+        if constexpr (READ) upd_bulk(sb + L.qr, qv + (size_t)head * DK, qbytes, bar);
         if (n > 0) {
             upd_bulk(sb + L.kr, kbuf + (size_t)head * W * DK, kbytes, bar);
             upd_bulk(sb + L.vr, vbuf + (size_t)head * W * dv, vbytes, bar);
@@ -410,8 +431,10 @@ update_window_persistent(ST *__restrict__ S, float *__restrict__ P, const float 
 
     // per-token scalars of the current head: lanes t and t + 32 of every warp
     auto load_scalars = [&](int w, float &a0, float &a1, float &b0, float &b1) {
-        const size_t base = (size_t)head_of(w) * W;
         a0 = a1 = b0 = b1 = 1.f;
+        const int hd = head_of(w);
+        if (SEQS && hd < 0) return;
+        const size_t base = (size_t)hd * W;
         if (KIND != KDA) {
             if (lane < n) a0 = abuf[base + lane];
             if (lane + 32 < n) a1 = abuf[base + lane + 32];
@@ -428,7 +451,7 @@ update_window_persistent(ST *__restrict__ S, float *__restrict__ P, const float 
     for (int w = w_begin, it = 0; w < w_end; ++w, ++it) {
         const int stage = it % ns;
         const int parity = (it / ns) & 1;
-        const int head = head_of(w), h = w / B;
+        const int head = head_of(w), h = w / NB;
         const char *sb = smem + L.stages + stage * L.stage_bytes;
         const bool landed = upd_wait(bars + 2 * stage, parity);
         // one decision for the whole CTA; the barrier also orders the previous
@@ -456,7 +479,7 @@ update_window_persistent(ST *__restrict__ S, float *__restrict__ P, const float 
             for (int i = tid; i < r * DK / 4; i += nthr) reinterpret_cast<float4 *>(sut)[i] = src[i];
             h_prev = h;
         }
-        if (qbytes) {
+        if constexpr (READ) {
             const QT *qr = reinterpret_cast<const QT *>(sb + L.qr);
             for (int i = tid; i < DK; i += nthr) sq[i] = ld1(qr + i);
         }
@@ -520,8 +543,9 @@ update_window_persistent(ST *__restrict__ S, float *__restrict__ P, const float 
         __syncthreads();  // the stage is consumed; the fp32 staging is ready
         if (tid == 0 && w + ns < w_end) issue(w + ns, stage);
 
-        apply_store_refresh<KIND, DK, ST, NC>(s, sk, su, sv, sg, sut, ss2, qbytes ? sq : nullptr, S, P, o, head, dv,
-                                              r, n, c0, l, lane);
+        if (!SEQS || head >= 0)  // CTA-uniform
+            apply_store_refresh<KIND, DK, ST, NC, READ>(s, sk, su, sv, sg, sut, ss2, sq, S, P, o, head, dv, r, n, c0, l,
+                                                        lane);
     }
 }
 
@@ -534,53 +558,66 @@ static size_t update_smem_bytes(const sketchssm_dims &d, int n) {
 
 int launch_update_window(const sketchssm_dims &d, void *S, float *P, const float *U, const void *k,
                          const void *v, const float *alpha, const float *beta, int n, const void *q, float *o,
-                         cudaStream_t stream) {
+                         const int *seqs, int n_seqs, int sm_share, cudaStream_t stream) {
     constexpr int LIMIT = 227 * 1024;
     return dispatch(d, [&](auto K, auto D, auto *sp, auto *qp) -> int {
         using ST = std::remove_pointer_t<decltype(sp)>;
         using QT = std::remove_pointer_t<decltype(qp)>;
         constexpr int KIND = decltype(K)::value, DK = decltype(D)::value;
-        const int NH = d.B * d.H;
-        // persistent kernel, state and tokens by bulk copies; one CTA per head if its layout does not fit
-        const int ns = PER_STAGES;
-        const PerLayout L = per_layout(KIND, DK, d.dv, d.r, n, sizeof(ST), sizeof(QT), ns);
-        if (L.total <= LIMIT) {
-            auto kern = update_window_persistent<KIND, DK, ST, QT, PER_NC>;
-            const int threads = d.dv * 8 / PER_NC;
+        const int NH = (seqs != nullptr ? n_seqs : d.B) * d.H;
+        if (NH == 0) return SKSSM_OK;
+        // the fused exact read is a separate instantiation: its code, even untaken, costs the plain
+        // update a few percent (measured)
+        auto run = [&](auto READc, auto SEQSc) -> int {
+            constexpr bool READ = decltype(READc)::value, SEQS = decltype(SEQSc)::value;
+            // persistent kernel, state and tokens by bulk copies; one CTA per head if its layout does not fit
+            const int ns = PER_STAGES;
+            const PerLayout L = per_layout(KIND, DK, d.dv, d.r, n, sizeof(ST), sizeof(QT), ns, READ);
+            if (L.total <= LIMIT) {
+                auto kern = update_window_persistent<KIND, DK, ST, QT, PER_NC, READ, SEQS>;
+                const int threads = d.dv * 8 / PER_NC;
+                static bool opted_in = false;
+                if (!opted_in) {
+                    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LIMIT) != cudaSuccess)
+                        return SKSSM_ERR_CUDA;
+                    opted_in = true;
+                }
+                int sms = 0, per_sm = 0;
+                if (sm_count(&sms) != SKSSM_OK ||
+                    blocks_per_sm(reinterpret_cast<const void *>(kern), threads, L.total, &per_sm) != SKSSM_OK)
+                    return SKSSM_ERR_CUDA;
+                if (per_sm >= 1) {
+                    if (sm_share > 0 && sm_share < per_sm) per_sm = sm_share;  // leave room for another kernel
+                    const int grid = NH < sms * per_sm ? NH : sms * per_sm;
+                    kern<<<grid, threads, L.total, stream>>>(static_cast<ST *>(S), P, U, static_cast<const QT *>(k),
+                                                             static_cast<const QT *>(v), alpha, beta,
+                                                             static_cast<const QT *>(q), o, d.B, d.H, d.dv, d.r, n,
+                                                             d.W, ns, seqs, n_seqs);
+                    return launch_status();
+                }
+            }
+            // one CTA per head
+            const int threads = d.dv * 8 / UPD_NC;
+            const size_t smem = update_smem_bytes(d, n);
+            if (smem > (size_t)LIMIT) return SKSSM_ERR_DIMS;
+            auto kern = update_window_kernel<KIND, DK, ST, QT, UPD_NC, READ, SEQS>;
             static bool opted_in = false;
             if (!opted_in) {
                 if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LIMIT) != cudaSuccess)
                     return SKSSM_ERR_CUDA;
                 opted_in = true;
             }
-            int sms = 0, per_sm = 0;
-            if (sm_count(&sms) != SKSSM_OK ||
-                blocks_per_sm(reinterpret_cast<const void *>(kern), threads, L.total, &per_sm) != SKSSM_OK)
-                return SKSSM_ERR_CUDA;
-            if (per_sm >= 1) {
-                const int grid = NH < sms * per_sm ? NH : sms * per_sm;
-                kern<<<grid, threads, L.total, stream>>>(static_cast<ST *>(S), P, U, static_cast<const QT *>(k),
-                                                         static_cast<const QT *>(v), alpha, beta,
-                                                         static_cast<const QT *>(q), o, d.B, d.H, d.dv, d.r, n, d.W,
-                                                         ns);
-                return launch_status();
-            }
+            kern<<<NH, threads, smem, stream>>>(static_cast<ST *>(S), P, U, static_cast<const QT *>(k),
+                                                static_cast<const QT *>(v), alpha, beta, static_cast<const QT *>(q),
+                                                o, d.B, d.H, d.dv, d.r, n, d.W, seqs, n_seqs);
+            return launch_status();
+        };
+        if (seqs != nullptr) {
+            if (q != nullptr) return run(std::true_type(), std::true_type());
+            return run(std::false_type(), std::true_type());
         }
-        // one CTA per head
-        const int threads = d.dv * 8 / UPD_NC;
-        const size_t smem = update_smem_bytes(d, n);
-        if (smem > (size_t)LIMIT) return SKSSM_ERR_DIMS;
-        auto kern = update_window_kernel<KIND, DK, ST, QT, UPD_NC>;
-        static bool opted_in = false;
-        if (!opted_in) {
-            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LIMIT) != cudaSuccess)
-                return SKSSM_ERR_CUDA;
-            opted_in = true;
-        }
-        kern<<<NH, threads, smem, stream>>>(static_cast<ST *>(S), P, U, static_cast<const QT *>(k),
-                                            static_cast<const QT *>(v), alpha, beta, static_cast<const QT *>(q), o,
-                                            d.B, d.H, d.dv, d.r, n, d.W);
-        return launch_status();
+        if (q != nullptr) return run(std::true_type(), std::false_type());
+        return run(std::false_type(), std::false_type());
     });
 }
 

@@ -17,8 +17,9 @@ from typing import Optional
 
 import torch
 
-from . import (sketchssm_decode_step, sketchssm_dims, sketchssm_fullread_decode, sketchssm_replay_decode_step,
-               sketchssm_update_window, sketchssm_update_window_read)
+from . import (sketchssm_decode_step, sketchssm_decode_step_seq, sketchssm_dims, sketchssm_fullread_decode,
+               sketchssm_replay_decode_step, sketchssm_update_window, sketchssm_update_window_read,
+               sketchssm_update_window_seqs)
 
 
 @dataclasses.dataclass
@@ -72,6 +73,36 @@ def sketch_window(d: sketchssm_dims, S, P, U, R, buf: WindowBuffer, out, n: Opti
                                      out[n - 1], stream)
     else:
         sketchssm_update_window(d, S, P, U, buf.k, buf.v, buf.alpha, buf.beta, n, stream)
+
+
+def stagger_plan(B: int, W: int, device="cuda"):
+    """Staggered windows: sequence b runs its windows with a phase of b mod W steps, so that at every
+    step about B/W sequences end a window.  For each step s of a W-step cycle: (j_seq, seqs), where
+    j_seq [B] int32 is each sequence's sketch step (0 for the sequences whose window ends at s) and
+    seqs int32 lists those sequences (their last step is read exactly by the window update)."""
+    b = torch.arange(B)
+    plan = []
+    for s in range(W):
+        j = (s + b) % W + 1
+        ends = j == W
+        plan.append((torch.where(ends, torch.zeros_like(j), j).to(torch.int32).to(device),
+                     b[ends].to(torch.int32).to(device)))
+    return plan
+
+
+def staggered_step(d: sketchssm_dims, S, P, U, R, buf: WindowBuffer, q, plan_s, out, sm_share=(0, 0),
+                   streams=(None, None)):
+    """One decode step of the staggered schedule: the sequences inside a window read the sketch
+    (q [B,H,dk] holds every sequence's query of this step; out [B,H,dv]), while the sequences whose
+    window ends are updated and read exactly.  The two launches touch disjoint sequences, so they
+    may run concurrently on two streams (streams = (decode, update)); sm_share caps each one's CTAs
+    per SM so that both fit on the GPU together."""
+    j_seq, seqs = plan_s
+    sketchssm_decode_step_seq(d, P, R, q, buf.k, buf.v, buf.alpha, buf.beta, j_seq, out, sm_share[0],
+                              streams[0])
+    if seqs.numel() > 0:
+        sketchssm_update_window_seqs(d, S, P, U, buf.k, buf.v, buf.alpha, buf.beta, d.W, seqs, q, out,
+                                     sm_share[1], streams[1])
 
 
 def replay_window(d: sketchssm_dims, S, buf: WindowBuffer, out, n: Optional[int] = None, stream=None):

@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--rank-avg", type=int, default=0,
+                    help="also time the sketch path with a rank per head: this average, the config's r the largest")
     ap.add_argument("--stagger-share", default="2,2",
                     help="CTAs per SM for the decode and update kernels of the staggered schedule")
     return ap.parse_args()
@@ -342,6 +344,12 @@ def run_ours(args):
     U = torch.empty(cfg.H, cfg.r, cfg.dk, device=dev)  # basis rows
     R = torch.empty(cfg.H, cfg.r, cfg.dk, device=dev)
     rs.sketchssm_calibrate_basis(dc, q_cal, S_cal, U, R)
+    if args.rank_avg:  # the same calibration data, ranks per head under an average-rank budget
+        Uk = torch.empty_like(U)
+        Rk = torch.empty_like(R)
+        head_rank = torch.empty(cfg.H, dtype=torch.int32, device=dev)
+        lam = torch.empty(cfg.H, cfg.r, dtype=torch.float64, device=dev)
+        rs.sketchssm_calibrate_basis_ranked(dc, q_cal, S_cal, args.rank_avg, Uk, Rk, head_rank, lam)
     del S_cal, P_cal, q_cal
 
     # NWIN distinct windows of decode tokens
@@ -368,6 +376,17 @@ def run_ours(args):
     fullread_window(d, Sf_a, toks[0], out_f)
     torch.cuda.synchronize()
     approx = float(torch.linalg.vector_norm((out - out_f).double()) / torch.linalg.vector_norm(out_f.double()))
+    if args.rank_avg:
+        S_k, P_k = S.clone(), torch.empty_like(P)
+        rs.sketchssm_update_window_ranked(d, S_k, P_k, Uk, head_rank, None, None, None, None, 0)
+        b0 = bufs[0]
+        for j in range(1, cfg.W + 1):
+            rs.sketchssm_decode_step_ranked(d, P_k, Rk, head_rank, b0.q[j - 1], b0.k, b0.v, b0.alpha, b0.beta, j,
+                                            out[j - 1])
+        torch.cuda.synchronize()
+        approx_k = float(torch.linalg.vector_norm((out - out_f).double()) /
+                         torch.linalg.vector_norm(out_f.double()))
+        del S_k
     S_a, P_a = S.clone(), P.clone()
     sketch_window(d, S_a, P_a, U, R, bufs[0], out, exact_last=True)
     torch.cuda.synchronize()
@@ -421,6 +440,20 @@ def run_ours(args):
         return fn
 
     g_st = [capture(stagger_cycle(b)) for b in bufs]
+    if args.rank_avg:  # the sketch path with a rank per head
+        Sk = S.clone()
+        Pk = torch.empty_like(P)
+        rs.sketchssm_update_window_ranked(d, Sk, Pk, Uk, head_rank, None, None, None, None, 0)
+
+        def ranked_window(b):
+            def fn():
+                for j in range(1, cfg.W + 1):
+                    rs.sketchssm_decode_step_ranked(d, Pk, Rk, head_rank, b.q[j - 1], b.k, b.v, b.alpha, b.beta, j,
+                                                    out[j - 1])
+                rs.sketchssm_update_window_ranked(d, Sk, Pk, Uk, head_rank, b.k, b.v, b.alpha, b.beta, cfg.W)
+            return fn
+
+        g_rk = [capture(ranked_window(b)) for b in bufs]
     # the ReplaySSM-style baseline: W full-state reads of the window-start state + one update (no sketch)
     Sr = S0.clone()
     g_rdec = [capture(lambda b=b: [rs.sketchssm_replay_decode_step(d, Sr, b.q[j - 1], b.k, b.v, b.alpha, b.beta,
@@ -510,6 +543,22 @@ def run_ours(args):
     barrier()
     clocks.mark(False)
     t_st = max_over_ranks(se0.elapsed_time(se1) / 1e3)
+
+    # --- rank per head
+    t_rk = None
+    if args.rank_avg:
+        for i in range(args.warmup):
+            g_rk[i % NWIN].replay()
+        barrier()
+        ke0, ke1 = ev(), ev()
+        clocks.mark(True)
+        ke0.record(stream)
+        for i in range(args.steps):
+            g_rk[i % NWIN].replay()
+        ke1.record(stream)
+        barrier()
+        clocks.mark(False)
+        t_rk = max_over_ranks(ke0.elapsed_time(ke1) / 1e3)
 
     # --- ReplaySSM-style baseline
     for i in range(args.warmup):
@@ -603,6 +652,13 @@ def run_ours(args):
             "replay_step_GBps": bm["replay_avg"] / (1e3 * t_rdec / (args.steps * cfg.W)) / 1e6,
             "algorithmic_bytes_per_token_step": bm["replay_step"] / tok_per_step,
             "sketch_speedup": value / whole_job_rate(args.steps * tok_per_step, world, t_r)},
+        **({"ranked": {
+            "value": whole_job_rate(args.steps * tok_per_step, world, t_rk), "unit": UNIT,
+            "ms_per_step": 1e3 * t_rk / args.steps, "r_avg": args.rank_avg, "r_max": cfg.r,
+            "ranks": head_rank.cpu().tolist(),
+            "schedule": "the sketch path with a rank per head (sketchssm_calibrate_basis_ranked, "
+                        "*_ranked kernels), same windows",
+            "approx_rel_l2_first_window": approx_k}} if args.rank_avg else {}),
         "staggered": {
             "value": whole_job_rate(args.steps * tok_per_step, world, t_st), "unit": UNIT,
             "ms_per_step": 1e3 * t_st / args.steps,
@@ -635,6 +691,8 @@ def run_ours(args):
     if rank == 0:
         print(json.dumps(line), flush=True)
     del g_dec, g_upd, g_full, g_x, g_rdec, g_rupd, g_st
+    if args.rank_avg:
+        del g_rk
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -210,6 +210,26 @@ int sketchssm_fullread_decode(const sketchssm_dims *dims, void *S, const void *q
                               void *stream);
 
 /*
+ * sketchssm_update_window_ranked, sketchssm_decode_step_ranked -- sketchssm_update_window
+ * and sketchssm_decode_step for a basis with a rank per head (as
+ * sketchssm_calibrate_basis_ranked makes it: U and R [H][r][dk] with rows
+ * m >= rank[h] zero).  The results equal the plain calls' on the same U and R;
+ * the window update skips the refresh arithmetic of the zero rows (and writes
+ * zero there), and the decode step reads the sketch columns m >= rank[h] only
+ * when rank[h] > 8, so that a head of rank <= 8 with r = 16 reads one 32-byte
+ * sector of each sketch row instead of two.
+ *   rank  in device [H] int32 (4-byte aligned); a value outside 0..r is counted by
+ *         sketchssm_device_error_count and clamped.
+ * Other arguments and errors as sketchssm_update_window / sketchssm_decode_step.
+ */
+int sketchssm_update_window_ranked(const sketchssm_dims *dims, void *S, float *P, const float *U,
+                                   const int32_t *rank, const void *k, const void *v, const float *alpha,
+                                   const float *beta, int n_tokens, void *stream);
+int sketchssm_decode_step_ranked(const sketchssm_dims *dims, const float *P, const float *R,
+                                 const int32_t *rank, const void *q, const void *k, const void *v,
+                                 const float *alpha, const float *beta, int j, float *o, void *stream);
+
+/*
  * sketchssm_replay_decode_step -- the second baseline: one decode step of a
  * buffered window that reads the full window-start state (ReplaySSM, as the
  * SketchSSM abstract and the digest bullet "Background" describe it: updates are
@@ -274,6 +294,34 @@ size_t sketchssm_calibrate_workspace_bytes(const sketchssm_dims *dims, int Nq, i
 int sketchssm_calibrate_basis(const sketchssm_dims *dims, const float *q_cal, int Nq,
                               const void *S_cal, int Ns, double ridge, float *U, float *R,
                               void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * sketchssm_calibrate_basis_ranked -- the offline calibration with a rank per head
+ * under an average-rank budget.  SketchSSM abstract and digest: the traffic
+ * reduction is quoted at an average sketch rank of 8, so ranks may differ across
+ * heads.  With the basis of sketchssm_calibrate_basis, head h's averaged read
+ * error at rank r is the sum of the eigenvalues of G^1/2 C G^1/2 past its r
+ * largest; the total error over heads is smallest when the budget of H * r_avg
+ * takes the largest of all heads' eigenvalues together, at most dims->r per head
+ * (ties: larger value, then lower head, then lower index).  Head h's basis is the
+ * first rank[h] rows of its rank-dims->r basis (U^T G U = I, so the same holds
+ * for R).
+ *   dims->r  r_max, the padded rank of U, R and P
+ *   r_avg    1..r_max, the average rank
+ *   U, R     out [H][r_max][dk] fp32, rows m >= rank[h] zero
+ *   rank     out device [H] int32
+ *   lam      out device [H][r_max] fp64: each head's r_max largest eigenvalues,
+ *            descending (8-byte aligned)
+ *   other arguments as sketchssm_calibrate_basis (same workspace size).
+ * With rows past a head's rank zero, every kernel of this library gives that
+ * head's rank-rank[h] results; the *_ranked calls also skip the work and the
+ * sketch traffic of those rows.
+ * Errors: as sketchssm_calibrate_basis; ERR_RANGE also for r_avg.
+ */
+int sketchssm_calibrate_basis_ranked(const sketchssm_dims *dims, const float *q_cal, int Nq,
+                                     const void *S_cal, int Ns, double ridge, int r_avg, float *U,
+                                     float *R, int32_t *rank, double *lam, void *workspace,
+                                     size_t workspace_bytes, void *stream);
 
 /*
  * sketchssm_calibrate_basis_noalloc -- sketchssm_calibrate_basis without a

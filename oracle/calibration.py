@@ -86,3 +86,58 @@ def objective(G: np.ndarray, C: np.ndarray, U: np.ndarray, R: np.ndarray) -> flo
     """Averaged squared read error tr(C (I - U R)^T G (I - U R)) of a basis/map pair."""
     E = np.eye(G.shape[0]) - U @ R
     return float(np.trace(C @ E.T @ G @ E))
+
+
+# ---------------------------------------------------------------------------
+# Heterogeneous per-head rank.  SketchSSM (arXiv 2609.33051v1) and the agihunt
+# digest quote the traffic reduction at an *average* sketch rank of 8, so ranks
+# may differ across heads.  The pages do not say how they are chosen; the reading
+# taken here: spend a total rank budget of H * r_avg where it removes the most
+# read error.  With the basis above, the averaged read error of head h at rank r
+# is sum_{i > r} lam_{h,i}, the eigenvalues of G^1/2 C G^1/2 past the r largest
+# (see residual_check in the tests), so the total error over heads is smallest
+# when the budget takes the H * r_avg largest eigenvalues of all heads together,
+# at most r_max per head.  Ties: larger value first, then lower head, then lower
+# index.  Head h's basis is the first r_h columns of its rank-r_max basis (U^T G U
+# is the identity, so its map R is the first r_h rows of the rank-r_max map).
+
+
+def spectrum_from_grams(G: np.ndarray, C: np.ndarray, ridge: float = 1e-8) -> np.ndarray:
+    """Eigenvalues of G^1/2 C G^1/2 (G with the ridge guard), in descending order."""
+    dk = G.shape[0]
+    G = G + ridge * (np.trace(G) / dk) * np.eye(dk)
+    Gh = _sym_power(G, 0.5)
+    A = Gh @ C @ Gh
+    A = 0.5 * (A + A.T)
+    return np.sort(np.linalg.eigvalsh(A))[::-1]
+
+
+def allocate_ranks(spectra: np.ndarray, r_avg: int, r_max: int) -> np.ndarray:
+    """Per-head ranks from per-head descending spectra [H, n] (n >= r_max): the H * r_avg
+    largest values over all heads, at most r_max per head."""
+    lam = np.asarray(spectra, dtype=np.float64)[:, :r_max]
+    H = lam.shape[0]
+    budget = H * r_avg
+    # candidates (value, head, index), ordered by value descending, then head, then index
+    order = sorted(((-lam[h, i], h, i) for h in range(H) for i in range(lam.shape[1])))
+    ranks = np.zeros(H, dtype=np.int64)
+    for _, h, _ in order[:budget]:
+        ranks[h] += 1
+    return ranks
+
+
+def calibrate_heads_ranked(S_cal: np.ndarray, q_cal: np.ndarray, r_avg: int, r_max: int,
+                           ridge: float = 1e-8):
+    """All heads with an average rank: U [H,dk,r_max] and R [H,r_max,dk] whose columns / rows past
+    head h's rank are zero, the ranks [H], and the spectra [H, dk]."""
+    S_cal = np.asarray(S_cal, dtype=np.float64)
+    q_cal = np.asarray(q_cal, dtype=np.float64)
+    H = S_cal.shape[1]
+    spectra = np.stack([spectrum_from_grams(gram_states(S_cal[:, h]), gram_queries(q_cal[h]), ridge)
+                        for h in range(H)])
+    ranks = allocate_ranks(spectra, r_avg, r_max)
+    U, R = calibrate_heads(S_cal, q_cal, r_max, ridge)
+    for h in range(H):
+        U[h][:, ranks[h]:] = 0.0
+        R[h][ranks[h]:, :] = 0.0
+    return U, R, ranks, spectra

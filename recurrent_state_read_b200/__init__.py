@@ -40,6 +40,9 @@ EXPORTS = (
     "sketchssm_calibrate_workspace_bytes",
     "sketchssm_calibrate_basis",
     "sketchssm_calibrate_basis_noalloc",
+    "sketchssm_calibrate_basis_ranked",
+    "sketchssm_update_window_ranked",
+    "sketchssm_decode_step_ranked",
     "sketchssm_device_error_count",
 )
 
@@ -88,10 +91,16 @@ def library() -> ctypes.CDLL:
         lib.sketchssm_calibrate_basis.argtypes = [D, P, i, P, i, ctypes.c_double, P, P, P,
                                                   ctypes.c_size_t, P]
         lib.sketchssm_calibrate_basis_noalloc.argtypes = [D, P, i, P, i, ctypes.c_double, P, P, P]
+        lib.sketchssm_calibrate_basis_ranked.argtypes = [D, P, i, P, i, ctypes.c_double, i, P, P, P, P, P,
+                                                         ctypes.c_size_t, P]
+        lib.sketchssm_update_window_ranked.argtypes = [D, P, P, P, P, P, P, P, P, i, P]
+        lib.sketchssm_decode_step_ranked.argtypes = [D, P, P, P, P, P, P, P, P, i, P, P]
         lib.sketchssm_device_error_count.argtypes = [i]
         lib.sketchssm_device_error_count.restype = i
         for f in ("sketchssm_update_window", "sketchssm_update_window_read", "sketchssm_decode_step",
-                  "sketchssm_replay_decode_step", "sketchssm_decode_step_seq", "sketchssm_update_window_seqs", "sketchssm_fullread_decode",
+                  "sketchssm_replay_decode_step", "sketchssm_decode_step_seq", "sketchssm_update_window_seqs",
+                  "sketchssm_calibrate_basis_ranked", "sketchssm_update_window_ranked",
+                  "sketchssm_decode_step_ranked", "sketchssm_fullread_decode",
                   "sketchssm_calibrate_basis", "sketchssm_calibrate_basis_noalloc"):
             getattr(lib, f).restype = i
         _lib = lib
@@ -264,6 +273,47 @@ def sketchssm_calibrate_basis(d: sketchssm_dims, q_cal, S_cal, U, R, workspace=N
         _ptr(S_cal, "S_cal", Ns * d.H * d.dv * d.dk, _dt(d.state_dtype)), int(Ns), float(ridge),
         _ptr(U, "U", d.H * d.dk * d.r, torch.float32), _ptr(R, "R", d.H * d.r * d.dk, torch.float32),
         _ptr(workspace, "workspace"), ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+        ctypes.c_void_p(_stream(stream))))
+
+
+def sketchssm_calibrate_basis_ranked(d: sketchssm_dims, q_cal, S_cal, r_avg: int, U, R, rank, lam,
+                                     workspace=None, ridge: float = 1e-8, stream=None):
+    """Offline basis with a rank per head under the average rank r_avg (d.r is the largest rank):
+    U, R [H,r,dk] with rows past rank[h] zero, rank int32 [H], lam float64 [H,r] (each head's r
+    largest eigenvalues, descending).  Workspace as sketchssm_calibrate_basis."""
+    Nq = q_cal.shape[1]
+    Ns = S_cal.shape[0]
+    need = sketchssm_calibrate_workspace_bytes(d, Nq, Ns)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q_cal.device)
+    _check("sketchssm_calibrate_basis_ranked", library().sketchssm_calibrate_basis_ranked(
+        ctypes.byref(d), _ptr(q_cal, "q_cal", d.H * Nq * d.dk, torch.float32), int(Nq),
+        _ptr(S_cal, "S_cal", Ns * d.H * d.dv * d.dk, _dt(d.state_dtype)), int(Ns), float(ridge), int(r_avg),
+        _ptr(U, "U", d.H * d.dk * d.r, torch.float32), _ptr(R, "R", d.H * d.r * d.dk, torch.float32),
+        _i32(rank, "rank", d.H), _ptr(lam, "lam", d.H * d.r, torch.float64),
+        _ptr(workspace, "workspace"), ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+        ctypes.c_void_p(_stream(stream))))
+
+
+def sketchssm_update_window_ranked(d: sketchssm_dims, S, P, U, rank, k, v, alpha, beta, n_tokens: int,
+                                   stream=None):
+    """sketchssm_update_window for a basis with a rank per head (rank int32 [H] on the device)."""
+    NH = d.B * d.H
+    toks = _token_ptrs(d, d.W, k, v, alpha, beta) if n_tokens > 0 else (None,) * 4
+    _check("sketchssm_update_window_ranked", library().sketchssm_update_window_ranked(
+        ctypes.byref(d), _ptr(S, "S", NH * d.dv * d.dk, _dt(d.state_dtype)),
+        _ptr(P, "P", NH * d.dv * d.r, torch.float32), _ptr(U, "U", d.H * d.dk * d.r, torch.float32),
+        _i32(rank, "rank", d.H), *toks, int(n_tokens), ctypes.c_void_p(_stream(stream))))
+
+
+def sketchssm_decode_step_ranked(d: sketchssm_dims, P, R, rank, q, k, v, alpha, beta, j: int, o, stream=None):
+    """sketchssm_decode_step for a basis with a rank per head (rank int32 [H] on the device)."""
+    NH = d.B * d.H
+    toks = _token_ptrs(d, d.W, k, v, alpha, beta)
+    _check("sketchssm_decode_step_ranked", library().sketchssm_decode_step_ranked(
+        ctypes.byref(d), _ptr(P, "P", NH * d.dv * d.r, torch.float32),
+        _ptr(R, "R", d.H * d.r * d.dk, torch.float32), _i32(rank, "rank", d.H),
+        _ptr(q, "q", NH * d.dk, _dt(d.qkv_dtype)), *toks, int(j), _ptr(o, "o", NH * d.dv, torch.float32),
         ctypes.c_void_p(_stream(stream))))
 
 

@@ -67,7 +67,7 @@ int sketchssm_update_window(const sketchssm_dims *d, void *S, float *P, const fl
     if (n_tokens > 0 && (rc = check_tokens(d, k, v, alpha, beta))) return rc;
     if (!aligned(S, 16) || !aligned(P, 16) || !aligned(U, 16)) return SKSSM_ERR_ALIGN;
     return launch_update_window(*d, S, P, P ? U : nullptr, k, v, alpha, beta, n_tokens, nullptr, nullptr, nullptr,
-                                0, 0, (cudaStream_t)stream);
+                                0, 0, nullptr, (cudaStream_t)stream);
 }
 
 int sketchssm_update_window_read(const sketchssm_dims *d, void *S, float *P, const float *U, const void *k,
@@ -80,7 +80,8 @@ int sketchssm_update_window_read(const sketchssm_dims *d, void *S, float *P, con
     if (n_tokens > 0 && (rc = check_tokens(d, k, v, alpha, beta))) return rc;
     if (!aligned(S, 16) || !aligned(P, 16) || !aligned(U, 16) || !aligned(q, 16) || !aligned(o, 16))
         return SKSSM_ERR_ALIGN;
-    return launch_update_window(*d, S, P, U, k, v, alpha, beta, n_tokens, q, o, nullptr, 0, 0, (cudaStream_t)stream);
+    return launch_update_window(*d, S, P, U, k, v, alpha, beta, n_tokens, q, o, nullptr, 0, 0, nullptr,
+                                (cudaStream_t)stream);
 }
 
 int sketchssm_decode_step(const sketchssm_dims *d, const float *P, const float *R, const void *q,
@@ -92,7 +93,7 @@ int sketchssm_decode_step(const sketchssm_dims *d, const float *P, const float *
     if (j < 1 || j > d->W) return SKSSM_ERR_RANGE;
     if ((rc = check_tokens(d, k, v, alpha, beta))) return rc;
     if (!aligned(P, 16) || !aligned(R, 16) || !aligned(q, 16) || !aligned(o, 16)) return SKSSM_ERR_ALIGN;
-    return launch_decode_step(*d, P, R, q, k, v, alpha, beta, j, nullptr, 0, o, (cudaStream_t)stream);
+    return launch_decode_step(*d, P, R, q, k, v, alpha, beta, j, nullptr, 0, nullptr, o, (cudaStream_t)stream);
 }
 
 int sketchssm_fullread_decode(const sketchssm_dims *d, void *S, const void *q, const void *k,
@@ -116,7 +117,7 @@ int sketchssm_decode_step_seq(const sketchssm_dims *d, const float *P, const flo
     if ((rc = check_tokens(d, k, v, alpha, beta))) return rc;
     if (!aligned(P, 16) || !aligned(R, 16) || !aligned(q, 16) || !aligned(o, 16) || !aligned(j_seq, 4))
         return SKSSM_ERR_ALIGN;
-    return launch_decode_step(*d, P, R, q, k, v, alpha, beta, d->W, j_seq, sm_share, o, (cudaStream_t)stream);
+    return launch_decode_step(*d, P, R, q, k, v, alpha, beta, d->W, j_seq, sm_share, nullptr, o, (cudaStream_t)stream);
 }
 
 int sketchssm_update_window_seqs(const sketchssm_dims *d, void *S, float *P, const float *U, const void *k,
@@ -132,7 +133,33 @@ int sketchssm_update_window_seqs(const sketchssm_dims *d, void *S, float *P, con
         !aligned(seqs, 4))
         return SKSSM_ERR_ALIGN;
     return launch_update_window(*d, S, P, P ? U : nullptr, k, v, alpha, beta, n_tokens, q, o, seqs, n_seqs, sm_share,
+                                nullptr, (cudaStream_t)stream);
+}
+
+int sketchssm_update_window_ranked(const sketchssm_dims *d, void *S, float *P, const float *U, const int32_t *rank,
+                                   const void *k, const void *v, const float *alpha, const float *beta, int n_tokens,
+                                   void *stream) {
+    int rc = check_dims(d);
+    if (rc) return rc;
+    if (!S || !P || !U || !rank) return SKSSM_ERR_NULL;
+    if (n_tokens < 0 || n_tokens > d->W) return SKSSM_ERR_RANGE;
+    if (n_tokens > 0 && (rc = check_tokens(d, k, v, alpha, beta))) return rc;
+    if (!aligned(S, 16) || !aligned(P, 16) || !aligned(U, 16) || !aligned(rank, 4)) return SKSSM_ERR_ALIGN;
+    return launch_update_window(*d, S, P, U, k, v, alpha, beta, n_tokens, nullptr, nullptr, nullptr, 0, 0, rank,
                                 (cudaStream_t)stream);
+}
+
+int sketchssm_decode_step_ranked(const sketchssm_dims *d, const float *P, const float *R, const int32_t *rank,
+                                 const void *q, const void *k, const void *v, const float *alpha, const float *beta,
+                                 int j, float *o, void *stream) {
+    int rc = check_dims(d);
+    if (rc) return rc;
+    if (!P || !R || !rank || !q || !o) return SKSSM_ERR_NULL;
+    if (j < 1 || j > d->W) return SKSSM_ERR_RANGE;
+    if ((rc = check_tokens(d, k, v, alpha, beta))) return rc;
+    if (!aligned(P, 16) || !aligned(R, 16) || !aligned(q, 16) || !aligned(o, 16) || !aligned(rank, 4))
+        return SKSSM_ERR_ALIGN;
+    return launch_decode_step(*d, P, R, q, k, v, alpha, beta, j, nullptr, 0, rank, o, (cudaStream_t)stream);
 }
 
 int sketchssm_replay_decode_step(const sketchssm_dims *d, const void *S, const void *q, const void *k, const void *v,
@@ -165,6 +192,24 @@ int sketchssm_calibrate_basis(const sketchssm_dims *d, const float *q_cal, int N
         !aligned(workspace, 256))
         return SKSSM_ERR_ALIGN;
     return launch_calibrate(*d, q_cal, Nq, S_cal, Ns, ridge, U, R, workspace, (cudaStream_t)stream);
+}
+
+int sketchssm_calibrate_basis_ranked(const sketchssm_dims *d, const float *q_cal, int Nq, const void *S_cal, int Ns,
+                                     double ridge, int r_avg, float *U, float *R, int32_t *rank, double *lam,
+                                     void *workspace, size_t workspace_bytes, void *stream) {
+    int rc = check_dims(d);
+    if (rc) return rc;
+    if (!q_cal || !S_cal || !U || !R || !rank || !lam) return SKSSM_ERR_NULL;
+    if (Nq < 1 || Ns < 1 || !(ridge >= 0.0) || r_avg < 1 || r_avg > d->r) return SKSSM_ERR_RANGE;
+    if ((int64_t)Ns * d->dv >= (int64_t)1 << 31 || (int64_t)Nq * d->H >= (int64_t)1 << 31)
+        return SKSSM_ERR_RANGE;
+    if (!workspace || workspace_bytes < calibrate_workspace_bytes(*d, Nq, Ns)) return SKSSM_ERR_WORKSPACE;
+    if (!aligned(q_cal, 16) || !aligned(S_cal, 16) || !aligned(U, 16) || !aligned(R, 16) ||
+        !aligned(workspace, 256) || !aligned(rank, 4) || !aligned(lam, 8))
+        return SKSSM_ERR_ALIGN;
+    rc = launch_calibrate(*d, q_cal, Nq, S_cal, Ns, ridge, U, R, workspace, (cudaStream_t)stream, lam);
+    if (rc != SKSSM_OK) return rc;
+    return launch_rank_basis(*d, r_avg, lam, U, R, rank, (cudaStream_t)stream);
 }
 
 }  // extern "C"

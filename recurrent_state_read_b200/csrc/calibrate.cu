@@ -86,7 +86,7 @@ __device__ double block_sum(double x, double *red) {
 template <int DK>
 __global__ void __launch_bounds__(BASIS_THREADS)
 basis_kernel(double *__restrict__ Gw, const double *__restrict__ Cw, double *__restrict__ Tw, int r,
-             double ridge, float *__restrict__ U, float *__restrict__ R) {
+             double ridge, float *__restrict__ U, float *__restrict__ R, double *__restrict__ lam) {
     constexpr int LD = DK + 1;  // padded row stride of the shared matrix
     extern __shared__ double sm[];
     double *A = sm;                   // [DK][LD]
@@ -235,6 +235,11 @@ basis_kernel(double *__restrict__ Gw, const double *__restrict__ Cw, double *__r
     }
     __syncthreads();
 
+    // the selected eigenvalues, descending (the ranked calibration compares them across heads)
+    if (lam != nullptr)
+        for (int m = tid; m < r; m += BASIS_THREADS) lam[(size_t)h * r + m] = A[sel[m] * LD + sel[m]];
+    __syncthreads();
+
     // 6. U = L^-T V_r (back substitution, one column per thread), R = V_r^T L^T
     double *X = A;  // reuse: [r][DK]
     for (int m = tid; m < r; m += BASIS_THREADS) {
@@ -259,6 +264,48 @@ basis_kernel(double *__restrict__ Gw, const double *__restrict__ Cw, double *__r
     }
 }
 
+// Per-head ranks under an average-rank budget: the budget takes the largest of all
+// heads' selected eigenvalues together (ties: lower head, then lower index), at most
+// r_max per head; head h's rank is the number of its values taken.  One CTA.
+__global__ void __launch_bounds__(1024)
+allocate_ranks_kernel(const double *__restrict__ lam, int H, int rmax, int budget, int *__restrict__ rank) {
+    for (int h = threadIdx.x; h < H; h += blockDim.x) rank[h] = 0;
+    __syncthreads();
+    const int n = H * rmax;
+    for (int c = threadIdx.x; c < n; c += blockDim.x) {
+        const double lc = lam[c];
+        int pos = 0;
+        for (int c2 = 0; c2 < n; ++c2) {
+            const double l2 = lam[c2];
+            pos += (l2 > lc) || (l2 == lc && c2 < c);
+        }
+        if (pos < budget) atomicAdd(&rank[c / rmax], 1);
+    }
+}
+
+// Rows m >= rank[h] of head h's basis rows U [H][r][dk] and map R [H][r][dk] set to zero.
+__global__ void mask_ranks_kernel(float *__restrict__ U, float *__restrict__ R, const int *__restrict__ rank, int H,
+                                  int r, int dk) {
+    const size_t n = (size_t)H * r * dk;
+    for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < n; idx += (size_t)gridDim.x * blockDim.x) {
+        const int m = (int)((idx / dk) % r), h = (int)(idx / ((size_t)r * dk));
+        if (m >= rank[h]) {
+            U[idx] = 0.f;
+            R[idx] = 0.f;
+        }
+    }
+}
+
+int launch_rank_basis(const sketchssm_dims &d, int r_avg, const double *lam, float *U, float *R, int *rank,
+                      cudaStream_t stream) {
+    allocate_ranks_kernel<<<1, 1024, 0, stream>>>(lam, d.H, d.r, d.H * r_avg, rank);
+    if (launch_status() != SKSSM_OK) return SKSSM_ERR_CUDA;
+    const size_t n = (size_t)d.H * d.r * d.dk;
+    const int grid = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+    mask_ranks_kernel<<<grid, 256, 0, stream>>>(U, R, rank, d.H, d.r, d.dk);
+    return launch_status();
+}
+
 size_t calibrate_workspace_bytes(const sketchssm_dims &d, int, int) {
     return 3 * (size_t)d.H * d.dk * d.dk * sizeof(double);
 }
@@ -270,7 +317,7 @@ static size_t basis_smem() {
 }
 
 int launch_calibrate(const sketchssm_dims &d, const float *q_cal, int Nq, const void *S_cal, int Ns,
-                     double ridge, float *U, float *R, void *workspace, cudaStream_t stream) {
+                     double ridge, float *U, float *R, void *workspace, cudaStream_t stream, double *lam) {
     double *G = static_cast<double *>(workspace);
     double *C = G + (size_t)d.H * d.dk * d.dk;
     double *T = C + (size_t)d.H * d.dk * d.dk;
@@ -293,7 +340,7 @@ int launch_calibrate(const sketchssm_dims &d, const float *q_cal, int Nq, const 
         if (cudaFuncSetAttribute(basis_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem) != cudaSuccess)
             return SKSSM_ERR_CUDA;
-        basis_kernel<DK><<<d.H, BASIS_THREADS, smem, stream>>>(G, C, T, d.r, ridge, U, R);
+        basis_kernel<DK><<<d.H, BASIS_THREADS, smem, stream>>>(G, C, T, d.r, ridge, U, R, lam);
         return launch_status();
     };
     if (d.dk == 64) return run(std::integral_constant<int, 64>());
@@ -305,7 +352,7 @@ int launch_calibrate(const sketchssm_dims &d, const float *q_cal, int Nq, const 
 // kernels as launch_calibrate, with every head-indexed pointer offset to h0.
 int launch_calibrate_heads(const sketchssm_dims &d, const float *q_cal, int Nq, const void *S_cal,
                            int Ns, double ridge, float *U, float *R, void *workspace, int h0, int hc,
-                           cudaStream_t stream) {
+                           cudaStream_t stream, double *lam) {
     double *G = static_cast<double *>(workspace);
     double *C = G + (size_t)hc * d.dk * d.dk;
     double *T = C + (size_t)hc * d.dk * d.dk;
@@ -330,7 +377,8 @@ int launch_calibrate_heads(const sketchssm_dims &d, const float *q_cal, int Nq, 
             return SKSSM_ERR_CUDA;
         basis_kernel<DK><<<hc, BASIS_THREADS, smem, stream>>>(G, C, T, d.r, ridge,
                                                                U + (size_t)h0 * DK * d.r,
-                                                               R + (size_t)h0 * d.r * DK);
+                                                               R + (size_t)h0 * d.r * DK,
+                                                               lam ? lam + (size_t)h0 * d.r : nullptr);
         return launch_status();
     };
     if (d.dk == 64) return run(std::integral_constant<int, 64>());

@@ -98,4 +98,34 @@ __device__ __forceinline__ void backward_chunk(const char *ks, const char *vs, c
     }
 }
 
+// acc[e] += sum_{mm < 8, m0 + mm < lim} P[c_e][m0 + mm] c[mm] for the lane's value channels
+// c_e = VPL lane + e (sketch rows of r floats at Ph), four columns at a time: one 16-byte
+// piece per row when r is a multiple of 4, else one column at a time.
+template <int VPL>
+__device__ __forceinline__ void sketch_block(const float *Ph, int r, int m0, int lim, const float (&c)[8],
+                                             float (&acc)[VPL], int lane) {
+#pragma unroll
+    for (int q = 0; q < 8; q += 4) {
+        if (m0 + q >= lim) break;  // warp-uniform
+        float pv[VPL][4];
+#pragma unroll
+        for (int e = 0; e < VPL; ++e) {
+            const float *row = Ph + (size_t)(lane * VPL + e) * r + m0 + q;
+            if ((r & 3) == 0) {
+                const float4 a = *reinterpret_cast<const float4 *>(row);
+                pv[e][0] = a.x; pv[e][1] = a.y; pv[e][2] = a.z; pv[e][3] = a.w;
+            } else {
+#pragma unroll
+                for (int mm = 0; mm < 4; ++mm) pv[e][mm] = m0 + q + mm < r ? row[mm] : 0.f;
+            }
+        }
+#pragma unroll
+        for (int mm = 0; mm < 4; ++mm)
+            if (m0 + q + mm < lim) {
+#pragma unroll
+                for (int e = 0; e < VPL; ++e) acc[e] = fmaf(pv[e][mm], c[q + mm], acc[e]);
+            }
+    }
+}
+
 }  // namespace skssm

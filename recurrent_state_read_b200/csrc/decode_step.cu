@@ -169,13 +169,7 @@ decode_step_kernel(const float *__restrict__ P, const float *__restrict__ R, con
 #pragma unroll
                 for (int e = 0; e < VPL; ++e) acc[e] = fmaf(pp[e][mm], c[mm], acc[e]);
         } else {
-#pragma unroll
-            for (int mm = 0; mm < DEC_RPRE; ++mm)
-                if (m0 + mm < r) {
-#pragma unroll
-                    for (int e = 0; e < VPL; ++e)
-                        acc[e] = fmaf(Ph[(size_t)(lane * VPL + e) * r + m0 + mm], c[mm], acc[e]);
-                }
+            sketch_block<VPL>(Ph, r, m0, r, c, acc, lane);
         }
     }
     float *oh = o + (size_t)head * DV + lane * VPL;
@@ -214,12 +208,13 @@ struct DecStage {
     __host__ __device__ static int bytes(int j) { return QB + tokens(j); }
 };
 
-template <int KIND, int DK, int DV, typename QT, bool JV>
+template <int KIND, int DK, int DV, typename QT, bool JV, bool RANKED>
 __global__ void __launch_bounds__(DEC_WARPS * 32)
 decode_step_persistent(const float *__restrict__ P, const float *__restrict__ R, const QT *__restrict__ qv,
                        const QT *__restrict__ kbuf, const QT *__restrict__ vbuf,
                        const float *__restrict__ abuf, const float *__restrict__ bbuf,
-                       float *__restrict__ o, int B, int H, int r, int j, int W, const int *__restrict__ jv) {
+                       float *__restrict__ o, int B, int H, int r, int j, int W, const int *__restrict__ jv,
+                       const int *__restrict__ rank) {
     using SL = DecSlots<KIND, DK, DV, QT>;
     using STG = DecStage<KIND, DK, DV, QT>;
     constexpr int KPL = DK / 32, VPL = DV / 32;
@@ -289,7 +284,7 @@ decode_step_persistent(const float *__restrict__ P, const float *__restrict__ R,
     if (++nb == B) { nb = 0; ++nh; }
     int j_n = JV && i0 + 1 < i1 ? step_of(nb) : 0;  // the step of the next head, one head ahead of its copies
 
-    int h_rows = -1;
+    int h_rows = -1, rh = r;  // rh: the rank of head index h_rows (rows past it are zero)
     float rr[DEC_RPRE][KPL];
     for (int i = i0, it = 0; i < i1; ++i, ++it) {
         const int s = it & 1;
@@ -313,6 +308,13 @@ decode_step_persistent(const float *__restrict__ P, const float *__restrict__ R,
                 }
             }
             h_rows = ch;
+            if constexpr (RANKED) {  // a rank outside 0..r is counted and clamped: no row past r is read
+                rh = rank[ch];
+                if (rh < 0 || rh > r) {
+                    if (lane == 0) atomicAdd(&g_device_error, 1u);
+                    rh = rh < 0 ? 0 : r;
+                }
+            }
         }
         // this head's group has landed (the next head's may still be in flight); the warp
         // barrier makes every lane's copies visible to the whole warp
@@ -341,7 +343,7 @@ decode_step_persistent(const float *__restrict__ P, const float *__restrict__ R,
 #pragma unroll
             for (int e = 0; e < VPL; ++e) acc[e] = ob[e];
 #pragma unroll 1
-            for (int m0 = 0; m0 < r; m0 += DEC_RPRE) {
+            for (int m0 = 0; m0 < rh; m0 += DEC_RPRE) {
                 float c[DEC_RPRE];
 #pragma unroll
                 for (int mm = 0; mm < DEC_RPRE; ++mm) {
@@ -349,7 +351,7 @@ decode_step_persistent(const float *__restrict__ P, const float *__restrict__ R,
                     if (m0 == 0) {
 #pragma unroll
                         for (int e = 0; e < KPL; ++e) c[mm] = fmaf(rr[mm][e], w[e], c[mm]);
-                    } else if (m0 + mm < r) {
+                    } else if (m0 + mm < rh) {
                         float rv[KPL];
                         load_n<KPL>(Rh + (size_t)(m0 + mm) * DK + lane * KPL, rv);
 #pragma unroll
@@ -357,16 +359,13 @@ decode_step_persistent(const float *__restrict__ P, const float *__restrict__ R,
                     }
                 }
                 warp_allreduce8(c, lane);
+                if (m0 == 0) {
 #pragma unroll
-                for (int mm = 0; mm < DEC_RPRE; ++mm) {
-                    if (m0 == 0) {
+                    for (int mm = 0; mm < DEC_RPRE; ++mm)
 #pragma unroll
                         for (int e = 0; e < VPL; ++e) acc[e] = fmaf(pp_c[e][mm], c[mm], acc[e]);
-                    } else if (m0 + mm < r) {
-#pragma unroll
-                        for (int e = 0; e < VPL; ++e)
-                            acc[e] = fmaf(Ph[(size_t)(lane * VPL + e) * r + m0 + mm], c[mm], acc[e]);
-                    }
+                } else {
+                    sketch_block<VPL>(Ph, r, m0, rh, c, acc, lane);
                 }
             }
             float *oh = o + (size_t)head * DV + lane * VPL;
@@ -389,7 +388,7 @@ decode_step_persistent(const float *__restrict__ P, const float *__restrict__ R,
 
 int launch_decode_step(const sketchssm_dims &d, const float *P, const float *R, const void *q,
                        const void *k, const void *v, const float *alpha, const float *beta, int j,
-                       const int *jv, int sm_share, float *o, cudaStream_t stream) {
+                       const int *jv, int sm_share, const int *rank, float *o, cudaStream_t stream) {
     if (jv != nullptr) j = d.W;  // per-sequence steps: size everything for the longest
     // the kernel does not touch the state: both state dtypes dispatch to the same instantiation
     return dispatch(d, [&](auto K, auto D, auto *, auto *qp) -> int {
@@ -405,8 +404,9 @@ int launch_decode_step(const sketchssm_dims &d, const float *P, const float *R, 
                 if (psmem <= 227 * 1024) {
                     // per-sequence steps are a separate instantiation: their checks cost the uniform
                     // step a few percent (measured)
-                    auto persist = [&](auto JVc) -> int {
-                        auto pk = decode_step_persistent<KIND, DK, DV, QT, decltype(JVc)::value>;
+                    auto persist = [&](auto JVc, auto RANKEDc) -> int {
+                        auto pk = decode_step_persistent<KIND, DK, DV, QT, decltype(JVc)::value,
+                                                         decltype(RANKEDc)::value>;
                         static bool p_opted_in = false;
                         if (!p_opted_in) {
                             if (cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
@@ -425,10 +425,12 @@ int launch_decode_step(const sketchssm_dims &d, const float *P, const float *R, 
                         const int pgrid = grid < sms * per_sm ? grid : sms * per_sm;
                         pk<<<pgrid, DEC_WARPS * 32, psmem, stream>>>(
                             P, R, static_cast<const QT *>(q), static_cast<const QT *>(k), static_cast<const QT *>(v),
-                            alpha, beta, o, d.B, d.H, d.r, j, d.W, jv);
+                            alpha, beta, o, d.B, d.H, d.r, j, d.W, jv, rank);
                         return launch_status();
                     };
-                    const int rc = jv != nullptr ? persist(std::true_type()) : persist(std::false_type());
+                    using T = std::true_type;
+                    using F = std::false_type;
+                    const int rc = jv != nullptr ? persist(T(), F()) : rank != nullptr ? persist(F(), T()) : persist(F(), F());
                     if (rc != 1) return rc;
                 }
             }

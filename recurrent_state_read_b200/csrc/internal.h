@@ -44,7 +44,7 @@ inline int launch_status() {
 
 int launch_update_window(const sketchssm_dims &d, void *S, float *P, const float *U, const void *k,
                          const void *v, const float *alpha, const float *beta, int n_tokens, const void *q, float *o,
-                         const int *seqs, int n_seqs, int sm_share, cudaStream_t stream);
+                         const int *seqs, int n_seqs, int sm_share, const int *rank, cudaStream_t stream);
 // Counts of bounded in-kernel waits that gave up (window update, decode step); reset clears them.
 int update_wait_giveups(bool reset, unsigned *count);
 int decode_wait_giveups(bool reset, unsigned *count);
@@ -104,13 +104,15 @@ int launch_fullread(const sketchssm_dims &d, void *S, const void *q, const void 
                     const float *alpha, const float *beta, float *o, cudaStream_t stream);
 int launch_decode_step(const sketchssm_dims &d, const float *P, const float *R, const void *q, const void *k,
                        const void *v, const float *alpha, const float *beta, int j, const int *jv, int sm_share,
-                       float *o, cudaStream_t stream);
+                       const int *rank, float *o, cudaStream_t stream);
 
 size_t calibrate_workspace_bytes(const sketchssm_dims &d, int Nq, int Ns);
+int launch_rank_basis(const sketchssm_dims &d, int r_avg, const double *lam, float *U, float *R, int *rank,
+                      cudaStream_t stream);
 int launch_calibrate(const sketchssm_dims &d, const float *q_cal, int Nq, const void *S_cal, int Ns,
-                     double ridge, float *U, float *R, void *workspace, cudaStream_t stream);
+                     double ridge, float *U, float *R, void *workspace, cudaStream_t stream, double *lam = nullptr);
 int launch_calibrate_heads(const sketchssm_dims &d, const float *q_cal, int Nq, const void *S_cal,
                            int Ns, double ridge, float *U, float *R, void *workspace, int h0, int hc,
-                           cudaStream_t stream);
+                           cudaStream_t stream, double *lam = nullptr);
 
 }  // namespace skssm

@@ -81,6 +81,17 @@ __device__ __forceinline__ void stage_rows(const T *__restrict__ src, size_t row
     }
 }
 
+// Rows of head index h's basis in use: rank[h], with a value outside 0..r counted as a
+// device error and clamped (so that no row past r is ever read).
+__device__ __forceinline__ int ranked_rows(const int *rank, int h, int r) {
+    const int v = rank[h];
+    if (v < 0 || v > r) {
+        if (threadIdx.x == 0) atomicAdd(&g_update_wait_giveups, 1u);
+        return v < 0 ? 0 : r;
+    }
+    return v;
+}
+
 // Steps shared by both window-update kernels, for one head whose state is in
 // registers: apply the n staged tokens in order, scale, round to the storage
 // type, store the state once, and refresh the sketch from the same registers.
@@ -89,7 +100,7 @@ __device__ __forceinline__ void apply_store_refresh(float (&s)[NC][DK / 8], cons
                                                     const float *sv, const float *sg, const float *sut,
                                                     const float *ss2, const float *sq, ST *__restrict__ S,
                                                     float *__restrict__ P, float *__restrict__ o, int head, int dv,
-                                                    int r, int n, int c0, int l, int lane) {
+                                                    int r, int r_used, int n, int c0, int l, int lane) {
     using TL = TileLayout<DK, ST>;
     constexpr int EPL = TL::EPL;
     const int cl = NC == 8 ? l : l >> 1;  // the column whose reduced values this lane holds
@@ -173,7 +184,7 @@ __device__ __forceinline__ void apply_store_refresh(float (&s)[NC][DK / 8], cons
 #pragma unroll
         for (int mm = 0; mm < 4; ++mm) {
             pm[mm] = 0.f;
-            if (m0 + mm < r) {
+            if (m0 + mm < r_used) {  // rows past a head's rank (zero basis rows) are written as zero
                 float uv[EPL];
                 lane_channels_smem<DK, ST>(sut + (m0 + mm) * DK, l, uv);
                 float d[NC];
@@ -284,7 +295,7 @@ update_window_kernel(ST *__restrict__ S, float *__restrict__ P, const float *__r
     }
     __syncthreads();
 
-    apply_store_refresh<KIND, DK, ST, NC, READ>(s, sk, su, sv, sg, sut, ss2, sq, S, P, o, head, dv, r, n,
+    apply_store_refresh<KIND, DK, ST, NC, READ>(s, sk, su, sv, sg, sut, ss2, sq, S, P, o, head, dv, r, r, n,
                                           c0, l, lane);
 }
 
@@ -355,13 +366,13 @@ __host__ __device__ inline PerLayout per_layout(int kind, int DK, int dv, int r,
     return L;
 }
 
-template <int KIND, int DK, typename ST, typename QT, int NC, bool READ, bool SEQS>
+template <int KIND, int DK, typename ST, typename QT, int NC, bool READ, bool SEQS, bool RANKED>
 __global__ void __launch_bounds__(256)
 update_window_persistent(ST *__restrict__ S, float *__restrict__ P, const float *__restrict__ U,
                          const QT *__restrict__ kbuf, const QT *__restrict__ vbuf,
                          const float *__restrict__ abuf, const float *__restrict__ bbuf,
                          const QT *__restrict__ qv, float *__restrict__ o, int B, int H, int dv, int r, int n, int W,
-                         int ns, const int *__restrict__ seqs, int n_seqs) {
+                         int ns, const int *__restrict__ seqs, int n_seqs, const int *__restrict__ rank) {
     using TL = TileLayout<DK, ST>;
     constexpr int EPL = TL::EPL;
     extern __shared__ __align__(128) float psm_f[];
@@ -544,7 +555,8 @@ update_window_persistent(ST *__restrict__ S, float *__restrict__ P, const float 
         if (tid == 0 && w + ns < w_end) issue(w + ns, stage);
 
         if (!SEQS || head >= 0)  // CTA-uniform
-            apply_store_refresh<KIND, DK, ST, NC, READ>(s, sk, su, sv, sg, sut, ss2, sq, S, P, o, head, dv, r, n, c0, l,
+            apply_store_refresh<KIND, DK, ST, NC, READ>(s, sk, su, sv, sg, sut, ss2, sq, S, P, o, head, dv, r,
+                                                        RANKED ? ranked_rows(rank, h, r) : r, n, c0, l,
                                                         lane);
     }
 }
@@ -558,7 +570,7 @@ static size_t update_smem_bytes(const sketchssm_dims &d, int n) {
 
 int launch_update_window(const sketchssm_dims &d, void *S, float *P, const float *U, const void *k,
                          const void *v, const float *alpha, const float *beta, int n, const void *q, float *o,
-                         const int *seqs, int n_seqs, int sm_share, cudaStream_t stream) {
+                         const int *seqs, int n_seqs, int sm_share, const int *rank, cudaStream_t stream) {
     constexpr int LIMIT = 227 * 1024;
     return dispatch(d, [&](auto K, auto D, auto *sp, auto *qp) -> int {
         using ST = std::remove_pointer_t<decltype(sp)>;
@@ -568,13 +580,14 @@ int launch_update_window(const sketchssm_dims &d, void *S, float *P, const float
         if (NH == 0) return SKSSM_OK;
         // the fused exact read is a separate instantiation: its code, even untaken, costs the plain
         // update a few percent (measured)
-        auto run = [&](auto READc, auto SEQSc) -> int {
+        auto run = [&](auto READc, auto SEQSc, auto RANKEDc) -> int {
             constexpr bool READ = decltype(READc)::value, SEQS = decltype(SEQSc)::value;
+            constexpr bool RANKED = decltype(RANKEDc)::value;
             // persistent kernel, state and tokens by bulk copies; one CTA per head if its layout does not fit
             const int ns = PER_STAGES;
             const PerLayout L = per_layout(KIND, DK, d.dv, d.r, n, sizeof(ST), sizeof(QT), ns, READ);
             if (L.total <= LIMIT) {
-                auto kern = update_window_persistent<KIND, DK, ST, QT, PER_NC, READ, SEQS>;
+                auto kern = update_window_persistent<KIND, DK, ST, QT, PER_NC, READ, SEQS, RANKED>;
                 const int threads = d.dv * 8 / PER_NC;
                 static bool opted_in = false;
                 if (!opted_in) {
@@ -592,7 +605,7 @@ int launch_update_window(const sketchssm_dims &d, void *S, float *P, const float
                     kern<<<grid, threads, L.total, stream>>>(static_cast<ST *>(S), P, U, static_cast<const QT *>(k),
                                                              static_cast<const QT *>(v), alpha, beta,
                                                              static_cast<const QT *>(q), o, d.B, d.H, d.dv, d.r, n,
-                                                             d.W, ns, seqs, n_seqs);
+                                                             d.W, ns, seqs, n_seqs, rank);
                     return launch_status();
                 }
             }
@@ -612,12 +625,15 @@ int launch_update_window(const sketchssm_dims &d, void *S, float *P, const float
                                                 o, d.B, d.H, d.dv, d.r, n, d.W, seqs, n_seqs);
             return launch_status();
         };
+        using T = std::true_type;
+        using F = std::false_type;
+        if (rank != nullptr) return run(F(), F(), T());  // the ranked update: no read, all sequences
         if (seqs != nullptr) {
-            if (q != nullptr) return run(std::true_type(), std::true_type());
-            return run(std::false_type(), std::true_type());
+            if (q != nullptr) return run(T(), T(), F());
+            return run(F(), T(), F());
         }
-        if (q != nullptr) return run(std::true_type(), std::false_type());
-        return run(std::false_type(), std::false_type());
+        if (q != nullptr) return run(T(), F(), F());
+        return run(F(), F(), F());
     });
 }
 

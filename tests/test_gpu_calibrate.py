@@ -77,3 +77,41 @@ def test_calibrate_bf16_states():
         Pi = U[h].T.double().cpu().numpy() @ R[h].double().cpu().numpy()
         Pi_ref = U_ref[h] @ R_ref[h]
         assert np.abs(Pi - Pi_ref).max() <= 1e-5 * max(1.0, np.abs(Pi_ref).max())
+
+
+@pytest.mark.parametrize("cid,r_max,r_avg", [(2, 16, 8), (1, 16, 8), (0, 8, 4)])
+def test_calibrate_ranked_matches_oracle(cid, r_max, r_avg):
+    """Ranked calibration: the GPU's eigenvalues against the oracle's spectra; the ranks, an integer
+    decision, bit for bit against the oracle's allocation applied to the GPU's eigenvalues; rows
+    past each rank zero; each head's projector against a rank-r_h oracle calibration."""
+    import recurrent_state_read_b200 as rs
+
+    cfg = wl.workload(cid, H=min(wl.CONFIGS[cid].H, 8), r=r_max, q_rank=12)
+    S_cal, q_cal = _cal_inputs(cfg, 16, 64, 1024)
+    # heads of different scales, so that the budget is spread unevenly
+    S_cal = S_cal * np.linspace(0.5, 2.0, cfg.H)[None, :, None, None]
+    q_np = q_cal.double().numpy() * np.linspace(0.5, 1.5, cfg.H)[:, None, None]
+    q_cal = torch.from_numpy(q_np).float()
+    d = rs.dims(cfg.kind, 16, cfg.H, cfg.dk, cfg.dv, r_max, cfg.W, torch.float32, cfg.torch_qkv_dtype)
+    S_gpu = to_gpu_state(S_cal.reshape(16 * cfg.H, cfg.dk, cfg.dv), 16, cfg.H)
+    U = torch.full((cfg.H, r_max, cfg.dk), float("nan"), device="cuda")
+    R = torch.full((cfg.H, r_max, cfg.dk), float("nan"), device="cuda")
+    rank = torch.full((cfg.H,), -1, dtype=torch.int32, device="cuda")
+    lam = torch.full((cfg.H, r_max), float("nan"), dtype=torch.float64, device="cuda")
+    rs.sketchssm_calibrate_basis_ranked(d, q_cal.cuda().contiguous(), S_gpu, r_avg, U, R, rank, lam)
+    torch.cuda.synchronize()
+    lam_g, rank_g = lam.cpu().numpy(), rank.cpu().numpy()
+    q_f = q_cal.double().numpy()
+    for h in range(cfg.H):
+        spec = cal.spectrum_from_grams(cal.gram_states(S_cal[:, h]), cal.gram_queries(q_f[h]))[:r_max]
+        np.testing.assert_allclose(lam_g[h], spec, rtol=1e-6, atol=1e-9 * spec[0])
+    assert rank_g.tolist() == cal.allocate_ranks(lam_g, r_avg, r_max).tolist()
+    assert rank_g.sum() == cfg.H * r_avg and len(set(rank_g.tolist())) > 1
+    Ug, Rg = U.transpose(1, 2).double().cpu().numpy(), R.double().cpu().numpy()
+    for h in range(cfg.H):
+        rh = int(rank_g[h])
+        assert np.all(Ug[h][:, rh:] == 0) and np.all(Rg[h][rh:] == 0)
+        if rh:
+            U_ref, R_ref = cal.calibrate(S_cal[:, h], q_f[h], rh)
+            Pi, Pi_ref = Ug[h] @ Rg[h], U_ref @ R_ref
+            assert np.abs(Pi - Pi_ref).max() <= 1e-5 * max(1.0, np.abs(Pi_ref).max()), h

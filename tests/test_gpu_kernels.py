@@ -326,3 +326,43 @@ def test_no_bounded_wait_gave_up():
     import recurrent_state_read_b200 as rs
 
     assert rs.sketchssm_device_error_count() == 0
+
+
+@pytest.mark.parametrize("kind", ["mamba2", "gdn", "kda"])
+def test_ranked_update_and_decode(kind):
+    """Rank per head (basis rows past rank[h] zero): the ranked window update and decode step give
+    the oracle's results for the zero-padded basis, i.e. each head's rank-r_h sketch read."""
+    import recurrent_state_read_b200 as rs
+
+    dk, dv, r, W = 128, 128 if kind != "mamba2" else 64, 16, 16
+    cfg, d, S0, U, R, tok = _setup(kind, dk, dv, r, W, torch.float32, torch.bfloat16, B=3, H=7, seed=8)
+    B, H = d.B, d.H
+    ranks = torch.tensor([0, 3, 8, 9, 16, 5, 12], dtype=torch.int32)
+    for h in range(H):
+        U[h][:, ranks[h]:] = 0
+        R[h][ranks[h]:] = 0
+    heads = np.arange(B * H)
+    Uh, Rh = oracle.per_head(U, H, heads), oracle.per_head(R, H, heads)
+    ft = flat_tokens(tok)
+    dev = to_device(tok)
+    win = to_window(dev)
+    S = to_gpu_state(S0, B, H)
+    P = torch.full((B, H, dv, r), float("nan"), device="cuda")
+    rk = ranks.cuda()
+    Ur = U.transpose(1, 2).contiguous().cuda()
+    rs.sketchssm_update_window_ranked(d, S, P, Ur, rk, win["k"], win["v"], win["alpha"], win["beta"], W)
+    torch.cuda.synchronize()
+    Sref, Pref = oracle.update_window(kind, S0, Uh, ft["k"], ft["v"], ft["alpha"], ft["beta"])
+    assert state_err(to_logical(S), Sref) <= STATE_TOL
+    assert state_err(P.reshape(B * H, dv, r).double().cpu().numpy(), Pref) <= STATE_TOL
+    assert torch.isfinite(P).all()
+    for j in (1, 9, W):
+        o = torch.full((B, H, dv), float("nan"), device="cuda")
+        rs.sketchssm_decode_step_ranked(d, P, R.cuda(), rk, dev["q"][j - 1], win["k"], win["v"], win["alpha"],
+                                        win["beta"], j, o)
+        torch.cuda.synchronize()
+        sl = slice(0, j)
+        ref = oracle.sketch_read(kind, Pref, Rh, ft["q"][j - 1], ft["k"][sl], ft["v"][sl], ft["alpha"][sl],
+                                 None if ft["beta"] is None else ft["beta"][sl])
+        assert rel_l2(o.reshape(B * H, dv).cpu(), ref) <= TIGHT_OUT, j
+    assert rs.sketchssm_device_error_count(1) == 0

@@ -7,6 +7,8 @@ direct minimisation over the calibration data, not through the Gram formula --
 that the oracle's basis minimises the averaged squared read error.
 """
 
+import itertools
+
 import numpy as np
 import pytest
 from scipy import optimize
@@ -140,3 +142,65 @@ def test_beats_query_pca_and_random_bases():
     assert ours <= _data_objective(S, q, Vt[:r].T) * (1 + 1e-12)
     for _ in range(20):
         assert ours <= _data_objective(S, q, rng.standard_normal((dk, r))) * (1 + 1e-12)
+
+
+# ---- heterogeneous per-head rank (average rank budget) ----------------------
+
+def _rand_grams(rng, dk, ns=40, nq=60):
+    S = rng.standard_normal((ns, dk, 5))
+    q = rng.standard_normal((nq, dk)) @ rng.standard_normal((dk, dk))
+    return cal.gram_states(S), cal.gram_queries(q)
+
+
+def test_residual_is_the_tail_of_the_spectrum():
+    """Closed form: at rank r the averaged read error of the basis equals the sum of the
+    eigenvalues of G^1/2 C G^1/2 past the r largest (pins spectrum_from_grams to objective)."""
+    rng = np.random.default_rng(21)
+    G, C = _rand_grams(rng, 7)
+    lam = cal.spectrum_from_grams(G, C, ridge=0.0)
+    assert np.all(np.diff(lam) <= 1e-12)
+    for r in range(0, 8):
+        if r == 0:
+            err = np.trace(C @ G)
+        else:
+            U, R = cal.basis_from_grams(G, C, r, ridge=0.0)
+            err = cal.objective(G, C, U, R)
+        assert err == pytest.approx(lam[r:].sum(), rel=1e-9, abs=1e-9 * lam.sum())
+
+
+def test_allocate_ranks_minimises_total_error_by_brute_force():
+    rng = np.random.default_rng(22)
+    for trial in range(20):
+        H, n, r_max = 3, 5, 4
+        r_avg = int(rng.integers(1, r_max + 1))
+        spectra = -np.sort(-rng.exponential(size=(H, n)) * rng.uniform(0.2, 3.0, size=(H, 1)), axis=1)
+        ranks = cal.allocate_ranks(spectra, r_avg, r_max)
+        assert ranks.sum() == H * r_avg and ranks.max() <= r_max
+        err = lambda rk: sum(spectra[h, rk[h]:].sum() for h in range(H))
+        best = min(err(rk) for rk in itertools.product(range(r_max + 1), repeat=H) if sum(rk) == H * r_avg)
+        assert err(ranks) == pytest.approx(best, rel=1e-12)
+
+
+def test_allocate_ranks_equal_spectra_and_cap():
+    lam = np.array([[5.0, 4.0, 3.0, 2.0, 1.0]] * 4)
+    assert cal.allocate_ranks(lam, 3, 5).tolist() == [3, 3, 3, 3]
+    dominant = np.array([[100.0, 90, 80, 70, 60], [1.0, 0.5, 0.2, 0.1, 0.05]])
+    assert cal.allocate_ranks(dominant, 2, 3).tolist() == [3, 1]  # capped at r_max = 3
+    assert cal.allocate_ranks(dominant, 2, 5).tolist() == [4, 0]
+
+
+def test_ranked_basis_is_the_truncated_full_basis():
+    rng = np.random.default_rng(23)
+    H, dk = 4, 6
+    S = rng.standard_normal((30, H, dk, 4)) * rng.uniform(0.3, 2.0, size=(1, H, 1, 1))
+    q = rng.standard_normal((H, 50, dk))
+    U, R, ranks, spectra = cal.calibrate_heads_ranked(S, q, 2, 4)
+    U4, R4 = cal.calibrate_heads(S, q, 4)
+    assert ranks.sum() == 2 * H
+    for h in range(H):
+        rh = ranks[h]
+        assert np.all(U[h][:, rh:] == 0) and np.all(R[h][rh:] == 0)
+        np.testing.assert_allclose(U[h][:, :rh], U4[h][:, :rh], rtol=0, atol=0)
+        if rh:  # the same projector as a rank-r_h calibration of that head alone
+            Ur, Rr = cal.calibrate(S[:, h], q[h], int(rh))
+            np.testing.assert_allclose(U[h] @ R[h], Ur @ Rr, atol=1e-9)

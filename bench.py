@@ -578,40 +578,81 @@ def run_ours(args):
     t_r = max_over_ranks(re_[0][0].elapsed_time(re_[-1][2]) / 1e3)
     t_rdec = sum(e[0].elapsed_time(e[1]) for e in re_) / 1e3
 
-    # --- end to end: window inputs from pinned host memory, outputs back to host
+    # --- end to end: window inputs from pinned host memory, outputs back to host.  As a serving
+    # loop would run it: the next window's inputs are copied in and the previous window's outputs
+    # copied out on two copy streams while the current window computes (NWIN input buffers, two
+    # output buffers; events order every reuse).
     e2e = None
     if not args.no_e2e:
         names = ("k", "v", "alpha", "beta", "q")
         host = []
         for b in bufs:
             host.append({n: getattr(b, n).cpu().pin_memory() for n in names if getattr(b, n) is not None})
-        out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        outs = [out, torch.empty_like(out)]
+        out_h = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
         h2d = sum(t.numel() * t.element_size() for t in host[0].values())
         d2h = out.numel() * out.element_size()
-        for i in range(min(args.warmup, 3)):
-            for n, t in host[i % NWIN].items():
-                getattr(bufs[i % NWIN], n).copy_(t, non_blocking=True)
-            g_dec[i % NWIN].replay()
-            g_upd[i % NWIN].replay()
-            out_h.copy_(out, non_blocking=True)
+
+        def dec_into(b, o):
+            return lambda: [rs.sketchssm_decode_step(d, P, R, b.q[j - 1], b.k, b.v, b.alpha, b.beta, j, o[j - 1])
+                            for j in range(1, cfg.W + 1)]
+
+        g_dec_e = [capture(dec_into(bufs[i], outs[i % 2])) for i in range(NWIN)]
+        up_s, down_s = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        h2d_ev = [torch.cuda.Event() for _ in range(NWIN)]
+        comp_ev = [torch.cuda.Event() for _ in range(NWIN)]
+        d2h_ev = [torch.cuda.Event() for _ in range(2)]
+
+        def copy_in(i):
+            b = i % NWIN
+            up_s.wait_event(comp_ev[b])  # the buffer's previous window has been computed
+            with torch.cuda.stream(up_s):
+                for n, t in host[b].items():
+                    getattr(bufs[b], n).copy_(t, non_blocking=True)
+            h2d_ev[b].record(up_s)
+
+        def compute(i):
+            b, o = i % NWIN, i % 2
+            stream.wait_event(h2d_ev[b])
+            stream.wait_event(d2h_ev[o])  # the output buffer has been copied out
+            g_dec_e[b].replay()
+            g_upd[b].replay()
+            comp_ev[b].record(stream)
+
+        def copy_out(i):
+            b, o = i % NWIN, i % 2
+            down_s.wait_event(comp_ev[b])
+            with torch.cuda.stream(down_s):
+                out_h[o].copy_(outs[o], non_blocking=True)
+            d2h_ev[o].record(down_s)
+
+        def run_e2e(n, start=None):
+            if start is not None:
+                up_s.wait_event(start)
+                down_s.wait_event(start)
+            copy_in(0)
+            for i in range(n):
+                compute(i)
+                if i + 1 < n:
+                    copy_in(i + 1)
+                copy_out(i)
+            stream.wait_event(d2h_ev[(n - 1) % 2])
+
+        run_e2e(min(args.warmup, 3))
         barrier()
         ee0, ee1 = ev(), ev()
         clocks.mark(True)
         ee0.record(stream)
-        for i in range(args.steps):
-            for n, t in host[i % NWIN].items():
-                getattr(bufs[i % NWIN], n).copy_(t, non_blocking=True)
-            g_dec[i % NWIN].replay()
-            g_upd[i % NWIN].replay()
-            out_h.copy_(out, non_blocking=True)
+        run_e2e(args.steps, ee0)
         ee1.record(stream)
         barrier()
         clocks.mark(False)
         t_e2e = max_over_ranks(ee0.elapsed_time(ee1) / 1e3)
         e2e = {"value": whole_job_rate(args.steps * cfg.B * cfg.W, world, t_e2e), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": 1e3 * t_e2e / args.steps,
-               "path": "python binding -> C ABI; pinned-host window inputs copied in and outputs copied "
-                       "out every step, inside the timed region"}
+               "path": "python binding -> C ABI; every window's inputs copied in from pinned host memory and "
+                       "its outputs copied out, inside the timed region, overlapped with the neighbouring "
+                       "windows' compute on two copy streams"}
     clk = clocks.stop()
 
     tok_per_step = cfg.B * cfg.W

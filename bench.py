@@ -440,6 +440,19 @@ def run_ours(args):
         return fn
 
     g_st = [capture(stagger_cycle(b)) for b in bufs]
+    g_wy = None
+    if cfg.kind != "mamba2" and cfg.W <= 32:  # the delta rules' decode step in WY form
+        Sw, Pw = S.clone(), P.clone()
+        Gw = rs.wy_gram_buffer(d, dev)
+
+        def wy_window(b):
+            def fn():
+                for j in range(1, cfg.W + 1):
+                    rs.sketchssm_decode_step_wy(d, Pw, R, b.q[j - 1], b.k, b.v, b.alpha, b.beta, j, Gw, out[j - 1])
+                rs.sketchssm_update_window(d, Sw, Pw, U, b.k, b.v, b.alpha, b.beta, cfg.W)
+            return fn
+
+        g_wy = [capture(wy_window(b)) for b in bufs]
     if args.rank_avg:  # the sketch path with a rank per head
         Sk = S.clone()
         Pk = torch.empty_like(P)
@@ -559,6 +572,22 @@ def run_ours(args):
         barrier()
         clocks.mark(False)
         t_rk = max_over_ranks(ke0.elapsed_time(ke1) / 1e3)
+
+    # --- decode steps in WY form
+    t_wy = None
+    if g_wy is not None:
+        for i in range(args.warmup):
+            g_wy[i % NWIN].replay()
+        barrier()
+        we0, we1 = ev(), ev()
+        clocks.mark(True)
+        we0.record(stream)
+        for i in range(args.steps):
+            g_wy[i % NWIN].replay()
+        we1.record(stream)
+        barrier()
+        clocks.mark(False)
+        t_wy = max_over_ranks(we0.elapsed_time(we1) / 1e3)
 
     # --- ReplaySSM-style baseline
     for i in range(args.warmup):
@@ -700,6 +729,11 @@ def run_ours(args):
             "schedule": "the sketch path with a rank per head (sketchssm_calibrate_basis_ranked, "
                         "*_ranked kernels), same windows",
             "approx_rel_l2_first_window": approx_k}} if args.rank_avg else {}),
+        **({"wy_decode": {
+            "value": whole_job_rate(args.steps * tok_per_step, world, t_wy), "unit": UNIT,
+            "ms_per_step": 1e3 * t_wy / args.steps,
+            "schedule": "the sketch path with the decode steps' backward pass in WY form "
+                        "(sketchssm_decode_step_wy, per-head Gram buffer)"}} if t_wy is not None else {}),
         "staggered": {
             "value": whole_job_rate(args.steps * tok_per_step, world, t_st), "unit": UNIT,
             "ms_per_step": 1e3 * t_st / args.steps,
@@ -731,7 +765,7 @@ def run_ours(args):
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del g_dec, g_upd, g_full, g_x, g_rdec, g_rupd, g_st
+    del g_dec, g_upd, g_full, g_x, g_rdec, g_rupd, g_st, g_wy
     if args.rank_avg:
         del g_rk
     if world > 1:

@@ -230,6 +230,26 @@ int sketchssm_decode_step_ranked(const sketchssm_dims *dims, const float *P, con
                                  const float *alpha, const float *beta, int j, float *o, void *stream);
 
 /*
+ * sketchssm_decode_step_wy -- sketchssm_decode_step for the delta rules (GDN, KDA)
+ * with the backward pass in WY / T-matrix form: the window's buffered keys have a
+ * Gram matrix (with the decays between them) that does not change while the
+ * window fills, so each step adds one column to a per-head buffer and solves a
+ * small triangular system against it instead of carrying the query back one
+ * token at a time.  Same results as sketchssm_decode_step (up to fp32 rounding).
+ *   G   in/out device [B][H][W][W4] fp32, W4 = W rounded up to a multiple of 4,
+ *       16-byte aligned, owned by the caller.  Step j writes row j-1 (entries
+ *       t < j-1) and reads rows 1..j-2, so within a window the steps must run in
+ *       order j = 1, 2, ..., each after the previous one (the same stream); the
+ *       buffer needs no initialisation and no reset between windows.
+ * SKSSM_MAMBA2 has no delta chain: the call is sketchssm_decode_step (G unused,
+ * may be NULL).  Requires W <= 32 (ERR_DIMS otherwise).
+ * Other arguments and errors as sketchssm_decode_step.
+ */
+int sketchssm_decode_step_wy(const sketchssm_dims *dims, const float *P, const float *R, const void *q,
+                             const void *k, const void *v, const float *alpha, const float *beta, int j,
+                             float *G, float *o, void *stream);
+
+/*
  * sketchssm_replay_decode_step -- the second baseline: one decode step of a
  * buffered window that reads the full window-start state (ReplaySSM, as the
  * SketchSSM abstract and the digest bullet "Background" describe it: updates are

@@ -43,6 +43,7 @@ EXPORTS = (
     "sketchssm_calibrate_basis_ranked",
     "sketchssm_update_window_ranked",
     "sketchssm_decode_step_ranked",
+    "sketchssm_decode_step_wy",
     "sketchssm_device_error_count",
 )
 
@@ -95,12 +96,13 @@ def library() -> ctypes.CDLL:
                                                          ctypes.c_size_t, P]
         lib.sketchssm_update_window_ranked.argtypes = [D, P, P, P, P, P, P, P, P, i, P]
         lib.sketchssm_decode_step_ranked.argtypes = [D, P, P, P, P, P, P, P, P, i, P, P]
+        lib.sketchssm_decode_step_wy.argtypes = [D, P, P, P, P, P, P, P, i, P, P, P]
         lib.sketchssm_device_error_count.argtypes = [i]
         lib.sketchssm_device_error_count.restype = i
         for f in ("sketchssm_update_window", "sketchssm_update_window_read", "sketchssm_decode_step",
                   "sketchssm_replay_decode_step", "sketchssm_decode_step_seq", "sketchssm_update_window_seqs",
                   "sketchssm_calibrate_basis_ranked", "sketchssm_update_window_ranked",
-                  "sketchssm_decode_step_ranked", "sketchssm_fullread_decode",
+                  "sketchssm_decode_step_ranked", "sketchssm_decode_step_wy", "sketchssm_fullread_decode",
                   "sketchssm_calibrate_basis", "sketchssm_calibrate_basis_noalloc"):
             getattr(lib, f).restype = i
         _lib = lib
@@ -315,6 +317,22 @@ def sketchssm_decode_step_ranked(d: sketchssm_dims, P, R, rank, q, k, v, alpha, 
         _ptr(R, "R", d.H * d.r * d.dk, torch.float32), _i32(rank, "rank", d.H),
         _ptr(q, "q", NH * d.dk, _dt(d.qkv_dtype)), *toks, int(j), _ptr(o, "o", NH * d.dv, torch.float32),
         ctypes.c_void_p(_stream(stream))))
+
+
+def wy_gram_buffer(d: sketchssm_dims, device="cuda"):
+    """The per-head Gram buffer of sketchssm_decode_step_wy: [B, H, W, W rounded up to 4] fp32."""
+    return torch.empty(d.B, d.H, d.W, (d.W + 3) // 4 * 4, dtype=torch.float32, device=device)
+
+
+def sketchssm_decode_step_wy(d: sketchssm_dims, P, R, q, k, v, alpha, beta, j: int, G, o, stream=None):
+    """Decode step j with the WY form of the backward pass; G from wy_gram_buffer, steps in order."""
+    NH = d.B * d.H
+    toks = _token_ptrs(d, d.W, k, v, alpha, beta)
+    _check("sketchssm_decode_step_wy", library().sketchssm_decode_step_wy(
+        ctypes.byref(d), _ptr(P, "P", NH * d.dv * d.r, torch.float32),
+        _ptr(R, "R", d.H * d.r * d.dk, torch.float32), _ptr(q, "q", NH * d.dk, _dt(d.qkv_dtype)),
+        *toks, int(j), _ptr(G, "G", NH * d.W * ((d.W + 3) // 4 * 4), torch.float32),
+        _ptr(o, "o", NH * d.dv, torch.float32), ctypes.c_void_p(_stream(stream))))
 
 
 def sketchssm_calibrate_basis_noalloc(d: sketchssm_dims, q_cal, S_cal, U, R, ridge: float = 1e-8, stream=None):

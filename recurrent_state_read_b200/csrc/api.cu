@@ -162,6 +162,20 @@ int sketchssm_decode_step_ranked(const sketchssm_dims *d, const float *P, const 
     return launch_decode_step(*d, P, R, q, k, v, alpha, beta, j, nullptr, 0, rank, o, (cudaStream_t)stream);
 }
 
+int sketchssm_decode_step_wy(const sketchssm_dims *d, const float *P, const float *R, const void *q, const void *k,
+                             const void *v, const float *alpha, const float *beta, int j, float *G, float *o,
+                             void *stream) {
+    int rc = check_dims(d);
+    if (rc) return rc;
+    if (d->W > 32) return SKSSM_ERR_DIMS;
+    if (!P || !R || !q || !o || (!G && d->kind != SKSSM_MAMBA2)) return SKSSM_ERR_NULL;
+    if (j < 1 || j > d->W) return SKSSM_ERR_RANGE;
+    if ((rc = check_tokens(d, k, v, alpha, beta))) return rc;
+    if (!aligned(P, 16) || !aligned(R, 16) || !aligned(q, 16) || !aligned(o, 16) || !aligned(G, 16))
+        return SKSSM_ERR_ALIGN;
+    return launch_decode_wy(*d, P, R, q, k, v, alpha, beta, j, G, o, (cudaStream_t)stream);
+}
+
 int sketchssm_replay_decode_step(const sketchssm_dims *d, const void *S, const void *q, const void *k, const void *v,
                                  const float *alpha, const float *beta, int j, float *o, void *stream) {
     int rc = check_dims(d);

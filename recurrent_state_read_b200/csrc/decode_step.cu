@@ -32,13 +32,11 @@
 namespace skssm {
 
 constexpr int DEC_WARPS = 4;  // one head per warp; small CTAs pack the SMs more tightly (measured)
-constexpr int DEC_RPRE = 8;   // sketch columns held in registers from the start; R rows per all-reduce
 constexpr unsigned DEC_WAIT_TRIES = 1u << 22;
 constexpr int DEC_PERSIST_MIN_WARPS = 12;  // fewest resident warps per SM for the pipelined kernel (measured crossover)
 
 __device__ unsigned g_device_error;
 
-__device__ __forceinline__ unsigned dec_smem(const void *p) { return (unsigned)__cvta_generic_to_shared(p); }
 
 __device__ __forceinline__ bool dec_wait(const uint64_t *bar, int phase) {
     for (unsigned it = 0; it < DEC_WAIT_TRIES; ++it) {

@@ -100,6 +100,9 @@ inline int read_counter(const T *symbol, bool reset, unsigned *count) {
 }
 int launch_replay_decode(const sketchssm_dims &d, const void *S, const void *q, const void *k, const void *v,
                          const float *alpha, const float *beta, int j, float *o, cudaStream_t stream);
+int launch_decode_wy(const sketchssm_dims &d, const float *P, const float *R, const void *q, const void *k,
+                     const void *v, const float *alpha, const float *beta, int j, float *G, float *o,
+                     cudaStream_t stream);
 int launch_fullread(const sketchssm_dims &d, void *S, const void *q, const void *k, const void *v,
                     const float *alpha, const float *beta, float *o, cudaStream_t stream);
 int launch_decode_step(const sketchssm_dims &d, const float *P, const float *R, const void *q, const void *k,

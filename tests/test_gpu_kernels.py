@@ -366,3 +366,54 @@ def test_ranked_update_and_decode(kind):
                                  None if ft["beta"] is None else ft["beta"][sl])
         assert rel_l2(o.reshape(B * H, dv).cpu(), ref) <= TIGHT_OUT, j
     assert rs.sketchssm_device_error_count(1) == 0
+
+
+WY_CASES = [
+    ("gdn", 128, 128, 8, 16, torch.bfloat16),
+    ("kda", 128, 128, 8, 16, torch.bfloat16),
+    ("gdn", 64, 64, 4, 5, torch.float32),       # odd window: padded Gram rows
+    ("kda", 64, 128, 16, 7, torch.float32),
+    ("gdn", 128, 64, 8, 32, torch.bfloat16),    # the longest window of the WY form
+    ("kda", 128, 128, 32, 32, torch.bfloat16),
+    ("mamba2", 128, 64, 8, 16, torch.bfloat16),  # no delta chain: the plain step
+]
+
+
+@pytest.mark.parametrize("case", WY_CASES, ids=[f"{c[0]}-dk{c[1]}-dv{c[2]}-r{c[3]}-W{c[4]}" for c in WY_CASES])
+def test_decode_step_wy(case):
+    """The WY form of the backward pass, steps 1..W in order on one Gram buffer (uninitialised:
+    NaN), against the oracle's token-by-token sketch read; the buffer's rows against the Gram
+    definition G_ut = sum_i k_t[i] k_u[i] a_{t+1}[i] ... a_u[i]."""
+    import recurrent_state_read_b200 as rs
+
+    kind, dk, dv, r, W, qdt = case
+    cfg, d, S0, U, R, tok = _setup(kind, dk, dv, r, W, torch.float32, qdt, seed=9)
+    B, H = d.B, d.H
+    g = torch.Generator().manual_seed(10)
+    P = torch.randn(B, H, dv, r, generator=g)
+    ft = flat_tokens(tok)
+    dev = to_device(tok)
+    win = to_window(dev)
+    Rh = oracle.per_head(R, H, np.arange(B * H))
+    G = rs.wy_gram_buffer(d)
+    G.fill_(float("nan"))
+    Pd, Rd = P.cuda(), R.cuda()
+    for j in range(1, W + 1):
+        o = torch.full((B, H, dv), float("nan"), device="cuda")
+        rs.sketchssm_decode_step_wy(d, Pd, Rd, dev["q"][j - 1], win["k"], win["v"], win["alpha"], win["beta"], j,
+                                    G, o)
+        torch.cuda.synchronize()
+        sl = slice(0, j)
+        ref = oracle.sketch_read(kind, P.reshape(B * H, dv, r), Rh, ft["q"][j - 1], ft["k"][sl], ft["v"][sl],
+                                 ft["alpha"][sl], None if ft["beta"] is None else ft["beta"][sl])
+        assert rel_l2(o.reshape(B * H, dv).cpu(), ref) <= TIGHT_OUT, j
+    if kind == "mamba2":
+        return
+    Gg = G.reshape(B * H, W, -1).double().cpu().numpy()
+    k, a = ft["k"], ft["alpha"]
+    for n in range(B * H):
+        for u in range(1, W):
+            for t in range(u):
+                dec = np.prod(a[t + 1:u + 1, n], axis=0) if kind == "kda" else np.prod(a[t + 1:u + 1, n])
+                ref_g = np.sum(k[t, n] * k[u, n] * dec)
+                assert abs(Gg[n, u, t] - ref_g) <= 1e-4 * max(1.0, abs(ref_g)), (n, u, t)

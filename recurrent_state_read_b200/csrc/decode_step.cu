@@ -33,6 +33,8 @@ namespace skssm {
 
 constexpr int DEC_WARPS = 4;  // one head per warp; small CTAs pack the SMs more tightly (measured)
 constexpr unsigned DEC_WAIT_TRIES = 1u << 22;
+constexpr int DEC_DEEP_STAGES = 2;       // shared-memory stages per warp of the deep-pipelined kernel (2 beat 3 and 4: more warps fit)
+constexpr int DEC_DEEP_MIN_WARPS = 8;     // fewest resident warps per SM for it
 constexpr int DEC_PERSIST_MIN_WARPS = 12;  // fewest resident warps per SM for the pipelined kernel (measured crossover)
 
 __device__ unsigned g_device_error;
@@ -384,6 +386,170 @@ decode_step_persistent(const float *__restrict__ P, const float *__restrict__ R,
     }
 }
 
+// ---------------------------------------------------------------------------
+// Deep-pipelined decode step (uniform step index, r = 8).  Everything a head needs arrives in one shared-memory
+// stage by cp.async -- query row, sketch rows, buffered k, v (and KDA decay) rows,
+// and the per-token scalars -- so a warp can keep NS - 1 heads in flight while it
+// computes one, with no register double-buffering.  One commit group per head; the
+// loop always commits exactly one group per iteration (empty past the warp's run),
+// so `cp.async.wait_group NS-1` always means "the current head has landed".
+//
+// The sketch rows are read per lane (lane l: rows VPL l .. VPL l + VPL-1, NP = VPL r / 4
+// sixteen-byte pieces).  Copied as they are, the lanes of a quarter-warp would hit the
+// same banks (a row pitch of 32 or 64 bytes), so the copy rotates each lane's pieces:
+// piece k of lane l goes to slot NP l + ((k + rot(l)) mod NP), rot(l) = l NP / 8 for
+// NP < 8 and l otherwise, which puts the eight lanes of a quarter-warp on distinct
+// 16-byte bank groups.
+// ---------------------------------------------------------------------------
+template <int KIND, int DK, int DV, typename QT>
+struct DeepStage {
+    using SL = DecSlots<KIND, DK, DV, QT>;
+    static constexpr int QB = DK * (int)sizeof(QT);
+    __host__ __device__ static int pbytes(int r) { return DV * r * 4; }
+    __host__ __device__ static int sbytes(int j) {  // per-token scalars: decay (not KDA), b (not Mamba-2)
+        return ((KIND != KDA ? 1 : 0) + (KIND != MAMBA2 ? 1 : 0)) * ((j * 4 + 15) & ~15);
+    }
+    __host__ __device__ static int bytes(int r, int j) {
+        return QB + pbytes(r) + j * (SL::KB + SL::VB + SL::AB) + sbytes(j);
+    }
+};
+
+__device__ __forceinline__ void cp_async4(char *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dec_smem(dst)), "l"(src) : "memory");
+}
+
+template <int NS>
+__device__ __forceinline__ void cp_async_wait_ns() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(NS - 1) : "memory");
+}
+
+template <int KIND, int DK, int DV, typename QT, int NS>
+__global__ void __launch_bounds__(DEC_WARPS * 32)
+decode_step_deep(const float *__restrict__ P, const float *__restrict__ R, const QT *__restrict__ qv,
+                 const QT *__restrict__ kbuf, const QT *__restrict__ vbuf, const float *__restrict__ abuf,
+                 const float *__restrict__ bbuf, float *__restrict__ o, int B, int H, int r, int j, int W) {
+    using SL = DecSlots<KIND, DK, DV, QT>;
+    using STG = DeepStage<KIND, DK, DV, QT>;
+    constexpr int KPL = DK / 32, VPL = DV / 32;
+    extern __shared__ __align__(16) char smem[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int NH = B * H;
+    const int sbytes = STG::bytes(r, j);
+    const int pbytes = STG::pbytes(r);
+    constexpr int NP = VPL * 2;                         // sixteen-byte sketch pieces per lane (r = 8)
+    const int rot = NP < 8 ? (lane * NP) >> 3 : lane;  // this lane's piece rotation
+    char *const stage0 = smem + (size_t)warp * NS * sbytes;
+
+    const int GW = gridDim.x * DEC_WARPS;
+    const int per = (NH + GW - 1) / GW;
+    const int i0 = (blockIdx.x * DEC_WARPS + warp) * per;
+    const int i1 = min(NH, i0 + per);
+    if (i0 >= i1) return;  // the whole warp; the kernel has no CTA-wide barrier
+
+    // the head run in (h, b) order: the issue cursor (ih, ib) runs NS - 1 heads ahead
+    int ih = i0 / B, ib = i0 - ih * B;
+    auto issue = [&](int i, int s) {  // one commit group, empty when i is past the run
+        if (i < i1) {
+            const int head = ib * H + ih;
+            char *sb = stage0 + s * sbytes;
+            char *qs = sb, *ps = qs + STG::QB, *ks = ps + pbytes, *vs = ks + j * SL::KB, *as = vs + j * SL::VB;
+            char *sc = as + j * SL::AB;
+            copy16(qs, qv + (size_t)head * DK, STG::QB, lane);
+            {  // sketch rows, each lane's pieces rotated (see above)
+                const char *src = reinterpret_cast<const char *>(P + (size_t)head * DV * r);
+                for (int pc = lane; pc < 32 * NP; pc += 32) {
+                    const int l = pc / NP, k = pc - l * NP;  // source piece k of lane l's rows
+                    const int rl = NP < 8 ? (l * NP) >> 3 : l;
+                    const int slot = l * NP + (k + rl) % NP;
+                    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dec_smem(ps + slot * 16)),
+                                 "l"(src + pc * 16)
+                                 : "memory");
+                }
+            }
+            copy16(ks, kbuf + (size_t)head * W * DK, j * SL::KB, lane);
+            copy16(vs, vbuf + (size_t)head * W * DV, j * SL::VB, lane);
+            if (KIND == KDA) copy16(as, abuf + (size_t)head * W * DK, j * SL::AB, lane);
+            if (lane < j) {
+                const int sstride = (j * 4 + 15) & ~15;
+                if (KIND != KDA) cp_async4(sc + lane * 4, abuf + (size_t)head * W + lane);
+                if (KIND != MAMBA2) cp_async4(sc + (KIND != KDA ? sstride : 0) + lane * 4, bbuf + (size_t)head * W + lane);
+            }
+            if (++ib == B) { ib = 0; ++ih; }
+        }
+        asm volatile("cp.async.commit_group;\n" ::: "memory");
+    };
+#pragma unroll
+    for (int s = 0; s < NS - 1; ++s) issue(i0 + s, s);
+
+    int ch = i0 / B, cb = i0 - ch * B;  // the head being computed
+    int h_rows = -1;
+    float rr[DEC_RPRE][KPL];
+    for (int i = i0, it = 0; i < i1; ++i, ++it) {
+        issue(i + NS - 1, (it + NS - 1) % NS);
+        const float *Rh = R + (size_t)ch * r * DK;
+        if (ch != h_rows) {  // warp-uniform
+#pragma unroll
+            for (int m = 0; m < DEC_RPRE; ++m) {
+                if (m < r) load_n<KPL>(Rh + (size_t)m * DK + lane * KPL, rr[m]);
+                else {
+#pragma unroll
+                    for (int e = 0; e < KPL; ++e) rr[m][e] = 0.f;
+                }
+            }
+            h_rows = ch;
+        }
+        cp_async_wait_ns<NS>();  // this head's group has landed (later heads may be in flight)
+        __syncwarp();
+        const char *sb = stage0 + (it % NS) * sbytes;
+        const char *qs = sb, *ps = qs + STG::QB, *ks = ps + pbytes, *vs = ks + j * SL::KB, *as = vs + j * SL::VB;
+        const float *sc = reinterpret_cast<const float *>(as + j * SL::AB);
+        const int sstride = ((j * 4 + 15) & ~15) / 4;
+        const float a_l = (KIND != KDA && lane < j) ? sc[lane] : 1.f;
+        const float b_l = (KIND != MAMBA2 && lane < j) ? sc[(KIND != KDA ? sstride : 0) + lane] : 1.f;
+        const int head = cb * H + ch;
+
+        float w[KPL], ob[VPL];
+        load_n<KPL>(reinterpret_cast<const QT *>(qs) + lane * KPL, w);
+#pragma unroll
+        for (int e = 0; e < VPL; ++e) ob[e] = 0.f;
+        float gsc = 1.f;
+        backward_chunk<KIND, DK, DV, QT>(ks, vs, as, j, a_l, b_l, w, ob, gsc, lane);
+        if (KIND != KDA) {
+#pragma unroll
+            for (int e = 0; e < KPL; ++e) w[e] *= gsc;
+        }
+        // c = R q~ (rows in registers), o = P c + o_buf with the lane's sketch rows from the stage
+        float c[DEC_RPRE];
+#pragma unroll
+        for (int mm = 0; mm < DEC_RPRE; ++mm) {
+            c[mm] = 0.f;
+#pragma unroll
+            for (int e = 0; e < KPL; ++e) c[mm] = fmaf(rr[mm][e], w[e], c[mm]);
+        }
+        warp_allreduce8(c, lane);
+        float acc[VPL];
+#pragma unroll
+        for (int e = 0; e < VPL; ++e) acc[e] = ob[e];
+        const float4 *pl = reinterpret_cast<const float4 *>(ps) + lane * NP;
+#pragma unroll
+        for (int k = 0; k < NP; ++k) {  // piece k: row VPL lane + k / 2, columns 4 (k mod 2) .. + 3
+            const float4 pv = pl[(k + rot) % NP];
+            const int e = k / 2, m = 4 * (k % 2);
+            acc[e] = fmaf(pv.x, c[m], acc[e]);
+            acc[e] = fmaf(pv.y, c[m + 1], acc[e]);
+            acc[e] = fmaf(pv.z, c[m + 2], acc[e]);
+            acc[e] = fmaf(pv.w, c[m + 3], acc[e]);
+        }
+        float *oh = o + (size_t)head * DV + lane * VPL;
+        if constexpr (VPL == 4) *reinterpret_cast<float4 *>(oh) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        else *reinterpret_cast<float2 *>(oh) = make_float2(acc[0], acc[1]);
+
+        __syncwarp();  // every lane is done with this stage before it is refilled
+        if (++cb == B) { cb = 0; ++ch; }
+    }
+    asm volatile("cp.async.wait_group 0;\n" ::: "memory");  // the empty groups past the run
+}
+
 int launch_decode_step(const sketchssm_dims &d, const float *P, const float *R, const void *q,
                        const void *k, const void *v, const float *alpha, const float *beta, int j,
                        const int *jv, int sm_share, const int *rank, float *o, cudaStream_t stream) {
@@ -397,6 +563,31 @@ int launch_decode_step(const sketchssm_dims &d, const float *P, const float *R, 
         auto go = [&](auto DVc) -> int {
             constexpr int DV = decltype(DVc)::value;
             // the persistent pipelined kernel, when a warp's two stages leave enough warps per SM
+            if (j <= 32 && d.r == 8 && jv == nullptr && rank == nullptr && sm_share == 0) {
+                const size_t dsmem = (size_t)DEC_WARPS * DEC_DEEP_STAGES * DeepStage<KIND, DK, DV, QT>::bytes(8, j);
+                if (dsmem <= 227 * 1024) {
+                    auto dk = decode_step_deep<KIND, DK, DV, QT, DEC_DEEP_STAGES>;
+                    static bool d_opted_in = false;
+                    if (!d_opted_in) {
+                        if (cudaFuncSetAttribute(dk, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+                            cudaSuccess)
+                            return SKSSM_ERR_CUDA;
+                        d_opted_in = true;
+                    }
+                    int sms = 0, per_sm = 0;
+                    if (sm_count(&sms) != SKSSM_OK ||
+                        blocks_per_sm(reinterpret_cast<const void *>(dk), DEC_WARPS * 32, dsmem, &per_sm) != SKSSM_OK)
+                        return SKSSM_ERR_CUDA;
+                    if (per_sm * DEC_WARPS >= DEC_DEEP_MIN_WARPS) {
+                        const int dgrid = grid < sms * per_sm ? grid : sms * per_sm;
+                        dk<<<dgrid, DEC_WARPS * 32, dsmem, stream>>>(P, R, static_cast<const QT *>(q),
+                                                                     static_cast<const QT *>(k),
+                                                                     static_cast<const QT *>(v), alpha, beta, o, d.B,
+                                                                     d.H, d.r, j, d.W);
+                        return launch_status();
+                    }
+                }
+            }
             if (j <= 32) {
                 const size_t psmem = (size_t)DEC_WARPS * 2 * DecStage<KIND, DK, DV, QT>::bytes(j);
                 if (psmem <= 227 * 1024) {

@@ -121,10 +121,19 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback (earlier copy measurement on this pool)"
 
 
-def csrc_hash():
+# the source files each profiled kernel is compiled from (a summary stays valid while they do not change)
+KERNEL_SOURCES = {
+    "decode_step": ("decode_step.cu", "decode_common.cuh", "common.cuh", "state_tile.cuh", "internal.h"),
+    "update_window": ("update_window.cu", "common.cuh", "state_tile.cuh", "internal.h"),
+}
+
+
+def csrc_hash(kernel=None):
+    """sha256 (16 hex digits) of a kernel's source files, or of every file under csrc/."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "recurrent_state_read_b200", "csrc")
-    for fn in sorted(os.listdir(d)):
+    names = KERNEL_SOURCES[kernel] if kernel else sorted(os.listdir(d))
+    for fn in names:
         with open(os.path.join(d, fn), "rb") as f:
             h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
@@ -141,7 +150,8 @@ def profiled_traffic(kernel_tag, cfg):
             if ":" in line and not line.startswith(" "):
                 k, v = line.split(":", 1)
                 kv[k.strip()] = v.strip()
-    if kv.get("csrc_sha256") != csrc_hash() or kv.get("workload_key") != workload_key(cfg):
+    kernel = "decode_step" if kernel_tag.startswith("decode_step") else "update_window"
+    if (kv.get("csrc_sha256") or "").split()[:1] != [csrc_hash(kernel)] or kv.get("workload_key") != workload_key(cfg):
         return None
     try:
         return float(kv["dram_bytes_per_launch_full_size"])

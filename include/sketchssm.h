@@ -284,6 +284,17 @@ int sketchssm_replay_decode_step(const sketchssm_dims *dims, const void *S, cons
 int sketchssm_device_error_count(int reset);
 
 /*
+ * sketchssm_selftest_wait_giveup -- makes the library's bounded-wait failure path
+ * run, for tests of failure detection: one warp waits on a shared-memory
+ * mbarrier that nothing arrives on, with the same wait every kernel of the
+ * library uses, bounded to `tries` polls (1..2^20); the wait gives up, counts
+ * itself in the sketchssm_device_error_count counter and the kernel returns,
+ * leaving the context usable.
+ * Errors: ERR_RANGE (tries), ERR_CUDA.
+ */
+int sketchssm_selftest_wait_giveup(unsigned tries, void *stream);
+
+/*
  * sketchssm_calibrate_workspace_bytes -- device workspace that
  * sketchssm_calibrate_basis needs for these sizes (0 if dims are invalid).
  */

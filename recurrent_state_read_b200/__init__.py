@@ -45,6 +45,7 @@ EXPORTS = (
     "sketchssm_decode_step_ranked",
     "sketchssm_decode_step_wy",
     "sketchssm_device_error_count",
+    "sketchssm_selftest_wait_giveup",
 )
 
 
@@ -98,6 +99,8 @@ def library() -> ctypes.CDLL:
         lib.sketchssm_decode_step_ranked.argtypes = [D, P, P, P, P, P, P, P, P, i, P, P]
         lib.sketchssm_decode_step_wy.argtypes = [D, P, P, P, P, P, P, P, i, P, P, P]
         lib.sketchssm_device_error_count.argtypes = [i]
+        lib.sketchssm_selftest_wait_giveup.argtypes = [ctypes.c_uint, P]
+        lib.sketchssm_selftest_wait_giveup.restype = i
         lib.sketchssm_device_error_count.restype = i
         for f in ("sketchssm_update_window", "sketchssm_update_window_read", "sketchssm_decode_step",
                   "sketchssm_replay_decode_step", "sketchssm_decode_step_seq", "sketchssm_update_window_seqs",
@@ -317,6 +320,13 @@ def sketchssm_decode_step_ranked(d: sketchssm_dims, P, R, rank, q, k, v, alpha, 
         _ptr(R, "R", d.H * d.r * d.dk, torch.float32), _i32(rank, "rank", d.H),
         _ptr(q, "q", NH * d.dk, _dt(d.qkv_dtype)), *toks, int(j), _ptr(o, "o", NH * d.dv, torch.float32),
         ctypes.c_void_p(_stream(stream))))
+
+
+def sketchssm_selftest_wait_giveup(tries: int = 1000, stream=None):
+    """Make the bounded-wait failure path run once (a wait that nothing satisfies): it is
+    counted in sketchssm_device_error_count and the context stays usable."""
+    _check("sketchssm_selftest_wait_giveup",
+           library().sketchssm_selftest_wait_giveup(int(tries), ctypes.c_void_p(_stream(stream))))
 
 
 def wy_gram_buffer(d: sketchssm_dims, device="cuda"):

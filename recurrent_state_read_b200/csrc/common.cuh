@@ -212,6 +212,35 @@ __device__ __forceinline__ float octet_sum(float x) {
     return x;
 }
 
+// ---- bounded mbarrier waits and bulk copies ---------------------------------
+// Every wait of the library on a shared-memory mbarrier polls a bounded number
+// of times; a wait that gives up returns false and the caller counts it
+// (sketchssm_device_error_count) instead of hanging the GPU.
+constexpr unsigned WAIT_TRIES = 1u << 22;
+
+__device__ __forceinline__ unsigned smem_u32(const void *p) { return (unsigned)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ bool mbar_wait(const uint64_t *bar, int parity, unsigned tries = WAIT_TRIES) {
+    for (unsigned it = 0; it < tries; ++it) {
+        unsigned done;
+        asm volatile(
+            "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }\n"
+            : "=r"(done)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+
+// One bulk copy global -> shared memory (TMA, no multicast), completing on bar.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, int bytes, const uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 // ---- L2 eviction priority hints ---------------------------------------------
 // The sketch P is re-read by every decode step of a window: it is written and
 // read with an evict-last policy so that it stays in L2 while the state and the

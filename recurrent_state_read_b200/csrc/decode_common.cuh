@@ -15,7 +15,7 @@ namespace skssm {
 
 constexpr int DEC_RPRE = 8;   // sketch columns held in registers from the start; R rows per all-reduce
 
-__device__ __forceinline__ unsigned dec_smem(const void *p) { return (unsigned)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ unsigned dec_smem(const void *p) { return smem_u32(p); }
 
 // Shared-memory slots of buffered tokens: 16 bytes (a barrier where one is used), then
 // jc k rows, jc v rows and (KDA) jc decay rows, each in its storage type.

@@ -32,7 +32,6 @@
 namespace skssm {
 
 constexpr int DEC_WARPS = 4;  // one head per warp; small CTAs pack the SMs more tightly (measured)
-constexpr unsigned DEC_WAIT_TRIES = 1u << 22;
 constexpr int DEC_DEEP_STAGES = 2;       // shared-memory stages per warp of the deep-pipelined kernel (2 beat 3 and 4: more warps fit)
 constexpr int DEC_DEEP_MIN_WARPS = 8;     // fewest resident warps per SM for it
 constexpr int DEC_PERSIST_MIN_WARPS = 12;  // fewest resident warps per SM for the pipelined kernel (measured crossover)
@@ -40,25 +39,6 @@ constexpr int DEC_PERSIST_MIN_WARPS = 12;  // fewest resident warps per SM for t
 __device__ unsigned g_device_error;
 
 
-__device__ __forceinline__ bool dec_wait(const uint64_t *bar, int phase) {
-    for (unsigned it = 0; it < DEC_WAIT_TRIES; ++it) {
-        unsigned done;
-        asm volatile(
-            "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }\n"
-            : "=r"(done)
-            : "r"(dec_smem(bar)), "r"(phase)
-            : "memory");
-        if (done) return true;
-    }
-    return false;
-}
-
-__device__ __forceinline__ void dec_bulk(void *dst, const void *src, int bytes, const uint64_t *bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
-                     dec_smem(dst)),
-                 "l"(src), "r"(bytes), "r"(dec_smem(bar))
-                 : "memory");
-}
 
 template <int KIND, int DK, int DV, typename QT>
 __global__ void __launch_bounds__(DEC_WARPS * 32)
@@ -126,13 +106,13 @@ decode_step_kernel(const float *__restrict__ P, const float *__restrict__ R, con
             asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(dec_smem(bar)),
                          "r"(nt * (SL::KB + SL::VB + SL::AB))
                          : "memory");
-            dec_bulk(ks, kbuf + row0 * DK, nt * SL::KB, bar);
-            dec_bulk(vs, vbuf + row0 * DV, nt * SL::VB, bar);
-            if (KIND == KDA) dec_bulk(as, abuf + row0 * DK, nt * SL::AB, bar);
+            bulk_g2s(ks, kbuf + row0 * DK, nt * SL::KB, bar);
+            bulk_g2s(vs, vbuf + row0 * DV, nt * SL::VB, bar);
+            if (KIND == KDA) bulk_g2s(as, abuf + row0 * DK, nt * SL::AB, bar);
         }
-        if (!dec_wait(bar, phase)) {
+        if (!mbar_wait(bar, phase)) {
             if (lane == 0) atomicAdd(&g_device_error, 1u);
-            dec_wait(bar, phase);  // give the copies in flight a last bounded chance to land
+            mbar_wait(bar, phase);  // give the copies in flight a last bounded chance to land
             return;
         }
         phase ^= 1;
@@ -648,6 +628,28 @@ int launch_decode_step(const sketchssm_dims &d, const float *P, const float *R, 
 }
 
 }  // namespace skssm
+
+namespace skssm {
+// The failure path every copy wait of the library shares, made to run: a bounded wait
+// on an mbarrier that nothing arrives on gives up after `tries` polls, is counted,
+// and the kernel returns, leaving the context usable.
+__global__ void wait_giveup_probe(unsigned tries) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_u32(&bar)) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    __syncwarp();
+    const bool landed = mbar_wait(&bar, 0, tries);
+    if (!landed && threadIdx.x == 0) atomicAdd(&g_device_error, 1u);
+}
+}  // namespace skssm
+
+extern "C" int sketchssm_selftest_wait_giveup(unsigned tries, void *stream) {
+    if (tries == 0 || tries > (1u << 20)) return SKSSM_ERR_RANGE;
+    skssm::wait_giveup_probe<<<1, 32, 0, (cudaStream_t)stream>>>(tries);
+    return skssm::launch_status();
+}
 
 int skssm::decode_wait_giveups(bool reset, unsigned *count) {
     return read_counter(&g_device_error, reset, count);

@@ -310,30 +310,6 @@ update_window_kernel(ST *__restrict__ S, float *__restrict__ P, const float *__r
 // (sketchssm_device_error_count) and the CTA returns.
 // ---------------------------------------------------------------------------
 
-constexpr unsigned UPD_WAIT_TRIES = 1u << 22;
-
-__device__ __forceinline__ unsigned upd_smem(const void *p) { return (unsigned)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ bool upd_wait(const uint64_t *bar, int parity) {
-    for (unsigned it = 0; it < UPD_WAIT_TRIES; ++it) {
-        unsigned done;
-        asm volatile(
-            "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }\n"
-            : "=r"(done)
-            : "r"(upd_smem(bar)), "r"(parity)
-            : "memory");
-        if (done) return true;
-    }
-    return false;
-}
-
-__device__ __forceinline__ void upd_bulk(void *dst, const void *src, int bytes, const uint64_t *bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
-                     upd_smem(dst)),
-                 "l"(src), "r"(bytes), "r"(upd_smem(bar))
-                 : "memory");
-}
-
 __host__ __device__ inline int up16(int x) { return (x + 15) & ~15; }
 
 // Byte offsets of the persistent kernel's shared memory (host and device agree).
@@ -415,25 +391,25 @@ update_window_persistent(ST *__restrict__ S, float *__restrict__ P, const float 
         uint64_t *bar = bars + 2 * stage;
         if (SEQS && head < 0) {  // nothing to copy: complete the stage's phase at once
             atomicAdd(&g_update_wait_giveups, 1u);
-            asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(upd_smem(bar)) : "memory");
+            asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
             return;
         }
         asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(upd_smem(bar)),
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)),
                      "r"(state_bytes + kbytes + vbytes + abytes + qbytes)
                      : "memory");
-        upd_bulk(sb + L.st, S + (size_t)head * dv * DK, state_bytes, bar);
-        if constexpr (READ) upd_bulk(sb + L.qr, qv + (size_t)head * DK, qbytes, bar);
+        bulk_g2s(sb + L.st, S + (size_t)head * dv * DK, state_bytes, bar);
+        if constexpr (READ) bulk_g2s(sb + L.qr, qv + (size_t)head * DK, qbytes, bar);
         if (n > 0) {
-            upd_bulk(sb + L.kr, kbuf + (size_t)head * W * DK, kbytes, bar);
-            upd_bulk(sb + L.vr, vbuf + (size_t)head * W * dv, vbytes, bar);
-            if (KIND == KDA) upd_bulk(sb + L.ar, abuf + (size_t)head * W * DK, abytes, bar);
+            bulk_g2s(sb + L.kr, kbuf + (size_t)head * W * DK, kbytes, bar);
+            bulk_g2s(sb + L.vr, vbuf + (size_t)head * W * dv, vbytes, bar);
+            if (KIND == KDA) bulk_g2s(sb + L.ar, abuf + (size_t)head * W * DK, abytes, bar);
         }
     };
 
     if (tid == 0) {
         for (int st = 0; st < ns; ++st)
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(upd_smem(bars + 2 * st)) : "memory");
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_u32(bars + 2 * st)) : "memory");
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
     __syncthreads();
@@ -464,14 +440,14 @@ update_window_persistent(ST *__restrict__ S, float *__restrict__ P, const float 
         const int parity = (it / ns) & 1;
         const int head = head_of(w), h = w / NB;
         const char *sb = smem + L.stages + stage * L.stage_bytes;
-        const bool landed = upd_wait(bars + 2 * stage, parity);
+        const bool landed = mbar_wait(bars + 2 * stage, parity);
         // one decision for the whole CTA; the barrier also orders the previous
         // head's reads of the fp32 staging before this head's writes
         if (__syncthreads_or(!landed)) {
             if (tid == 0) {  // count the give-up, then drain the copies still in flight (bounded)
                 atomicAdd(&g_update_wait_giveups, 1u);
                 for (int k2 = 0; k2 < ns && w + k2 < w_end; ++k2)
-                    upd_wait(bars + 2 * ((it + k2) % ns), ((it + k2) / ns) & 1);
+                    mbar_wait(bars + 2 * ((it + k2) % ns), ((it + k2) / ns) & 1);
             }
             __syncthreads();
             return;

@@ -95,6 +95,8 @@ def test_validation_codes(rs):
     assert ds(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, FAKE, None) == -3
     assert ds(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 17, FAKE, None) == -3
     assert ds(ctypes.byref(d), FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, 3, FAKE, None) == -1
+    assert lib.sketchssm_selftest_wait_giveup(0, None) == -3
+    assert lib.sketchssm_selftest_wait_giveup((1 << 20) + 1, None) == -3
     rp = lib.sketchssm_replay_decode_step
     assert rp(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, FAKE, None) == -3
     assert rp(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 17, FAKE, None) == -3

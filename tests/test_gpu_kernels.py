@@ -417,3 +417,25 @@ def test_decode_step_wy(case):
                 dec = np.prod(a[t + 1:u + 1, n], axis=0) if kind == "kda" else np.prod(a[t + 1:u + 1, n])
                 ref_g = np.sum(k[t, n] * k[u, n] * dec)
                 assert abs(Gg[n, u, t] - ref_g) <= 1e-4 * max(1.0, abs(ref_g)), (n, u, t)
+
+
+def test_bounded_wait_gives_up_and_the_context_survives():
+    """Failure detection without a GPU fault: a bounded wait that nothing satisfies gives up, is
+    counted, and the next real kernel runs normally."""
+    import recurrent_state_read_b200 as rs
+
+    torch.cuda.synchronize()
+    rs.sketchssm_device_error_count(1)  # start from zero
+    rs.sketchssm_selftest_wait_giveup(1000)
+    assert rs.sketchssm_device_error_count(1) == 1
+    assert rs.sketchssm_device_error_count(0) == 0  # reset took
+    kind, dk, dv, r, W, sdt, qdt = CASES[1]
+    cfg, d, S0, U, R, tok = _setup(kind, dk, dv, r, W, sdt, qdt, seed=12)
+    dev = to_device(tok)
+    win = to_window(dev)
+    P = torch.randn(d.B, d.H, dv, r, device="cuda")
+    o = torch.full((d.B, d.H, dv), float("nan"), device="cuda")
+    rs.sketchssm_decode_step(d, P, R.cuda(), dev["q"][3], win["k"], win["v"], win["alpha"], win["beta"], 4, o)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o).all()
+    assert rs.sketchssm_device_error_count(1) == 0

@@ -242,25 +242,14 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, int bytes, 
 }
 
 // ---- L2 eviction priority hints ---------------------------------------------
-// The sketch P is re-read by every decode step of a window: it is written and
-// read with an evict-last policy so that it stays in L2 while the state and the
-// buffered tokens stream past.
+// The sketch P is re-read by every decode step of a window: the window update
+// writes it with an evict-last policy so that it stays in L2 while the state
+// streams past (the decode steps read it with plain loads: an evict-last read
+// measured slower on the Mamba-2 workload).
 __device__ __forceinline__ uint64_t l2_evict_last_policy() {
     uint64_t pol;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
     return pol;
-}
-__device__ __forceinline__ float4 ld_keep(const float *p, uint64_t pol) {
-    float4 a;
-    asm volatile("ld.global.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
-                 : "=f"(a.x), "=f"(a.y), "=f"(a.z), "=f"(a.w)
-                 : "l"(p), "l"(pol));
-    return a;
-}
-__device__ __forceinline__ float ld_keep1(const float *p, uint64_t pol) {
-    float a;
-    asm volatile("ld.global.L2::cache_hint.f32 %0, [%1], %2;" : "=f"(a) : "l"(p), "l"(pol));
-    return a;
 }
 __device__ __forceinline__ void st_keep(float *p, float4 a, uint64_t pol) {
     asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "f"(a.x), "f"(a.y),

@@ -13,19 +13,22 @@
 // (q~ = M_1^T ... M_j^T q) and collects their exact contribution o_buf.  The
 // sketch replaces S0^T q~ by P (R q~).  Nothing is written to S.
 //
-// One warp per head (heads in (h, b) order, so a CTA's warps share R rows).
-// A decode step is one memory round trip per head: the head's buffered k and v
-// (and KDA decay) rows are contiguous blocks of the head-major window buffer
-// and arrive by TMA bulk copies into the warp's shared-memory slots, while the
-// query, the per-token scalars (one token per lane) and the first eight sketch
-// columns are loaded into registers at the same time.  The backward pass then
-// runs from shared memory: per token one warp reduction for k . w and one axpy.
-// Scalar decay is kept as a running scale next to the carried query (w = g w^),
-// so Mamba-2's dot products do not depend on each other and eight of them share
-// one warp all-reduce.  The coefficient rows R (the same for every b) are read
-// after the pass, from L1/L2, so that they hold no registers while the copies
-// are in flight: 64 registers per thread keep eight 4-warp CTAs on an SM.  The
-// wait on the copies is bounded: a give-up is counted in a device flag
+// Three kernels, one warp per head each, heads in (h, b) order (a CTA's warps share R
+// rows); the launcher takes the first that applies:
+//  - decode_step_deep (r = 8, one step index for all heads, at least 8 resident warps):
+//    persistent warps, the whole per-head working set staged by cp.async, two stages;
+//  - decode_step_persistent (per-sequence steps, per-head ranks, other r; at least 12
+//    resident warps): persistent warps, token rows staged by cp.async, sketch columns
+//    and per-token scalars prefetched into registers one head ahead;
+//  - decode_step_kernel (the rest: long windows, KDA's wide token rows): one head per
+//    warp, the head's buffered rows by TMA bulk copies on a bounded mbarrier wait, in
+//    chunks of up to 32 tokens, while the query, the per-token scalars and the first
+//    eight sketch columns load into registers; R rows are read after the backward pass
+//    from L1/L2 (64 registers: eight 4-warp CTAs per SM).
+// All three run the same backward pass (decode_common.cuh): per token one warp
+// reduction for k . w and one axpy; scalar decay is kept as a running scale next to the
+// carried query (w = g w^), so Mamba-2's dots do not depend on each other and eight of
+// them share one warp all-reduce.  A bounded wait that gives up is counted
 // (sketchssm_device_error_count) and the warp returns.
 #include "decode_common.cuh"
 

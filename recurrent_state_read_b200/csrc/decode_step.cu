@@ -388,7 +388,10 @@ template <int KIND, int DK, int DV, typename QT>
 struct DeepStage {
     using SL = DecSlots<KIND, DK, DV, QT>;
     static constexpr int QB = DK * (int)sizeof(QT);
-    __host__ __device__ static int pbytes(int r) { return DV * r * 4; }
+    // dv = 64: a lane's two sketch rows (32 bytes) go straight to registers at the start of the
+    // head, under the backward pass; dv = 128: its 64 bytes are staged (registers measured slower)
+    static constexpr bool P_IN_REGS = DV == 64;
+    __host__ __device__ static int pbytes(int r) { return P_IN_REGS ? 0 : DV * r * 4; }
     __host__ __device__ static int sbytes(int j) {  // per-token scalars: decay (not KDA), b (not Mamba-2)
         return ((KIND != KDA ? 1 : 0) + (KIND != MAMBA2 ? 1 : 0)) * ((j * 4 + 15) & ~15);
     }
@@ -438,7 +441,7 @@ decode_step_deep(const float *__restrict__ P, const float *__restrict__ R, const
             char *qs = sb, *ps = qs + STG::QB, *ks = ps + pbytes, *vs = ks + j * SL::KB, *as = vs + j * SL::VB;
             char *sc = as + j * SL::AB;
             copy16(qs, qv + (size_t)head * DK, STG::QB, lane);
-            {  // sketch rows, each lane's pieces rotated (see above)
+            if (!STG::P_IN_REGS) {  // sketch rows, each lane's pieces rotated (see above)
                 const char *src = reinterpret_cast<const char *>(P + (size_t)head * DV * r);
                 for (int pc = lane; pc < 32 * NP; pc += 32) {
                     const int l = pc / NP, k = pc - l * NP;  // source piece k of lane l's rows
@@ -490,6 +493,12 @@ decode_step_deep(const float *__restrict__ P, const float *__restrict__ R, const
         const float a_l = (KIND != KDA && lane < j) ? sc[lane] : 1.f;
         const float b_l = (KIND != MAMBA2 && lane < j) ? sc[(KIND != KDA ? sstride : 0) + lane] : 1.f;
         const int head = cb * H + ch;
+        float4 pr[STG::P_IN_REGS ? NP : 1];
+        if constexpr (STG::P_IN_REGS) {
+            const float4 *pg = reinterpret_cast<const float4 *>(P + (size_t)head * DV * 8) + lane * NP;
+#pragma unroll
+            for (int k = 0; k < NP; ++k) pr[k] = pg[k];
+        }
 
         float w[KPL], ob[VPL];
         load_n<KPL>(reinterpret_cast<const QT *>(qs) + lane * KPL, w);
@@ -516,7 +525,7 @@ decode_step_deep(const float *__restrict__ P, const float *__restrict__ R, const
         const float4 *pl = reinterpret_cast<const float4 *>(ps) + lane * NP;
 #pragma unroll
         for (int k = 0; k < NP; ++k) {  // piece k: row VPL lane + k / 2, columns 4 (k mod 2) .. + 3
-            const float4 pv = pl[(k + rot) % NP];
+            const float4 pv = STG::P_IN_REGS ? pr[k] : pl[(k + rot) % NP];
             const int e = k / 2, m = 4 * (k % 2);
             acc[e] = fmaf(pv.x, c[m], acc[e]);
             acc[e] = fmaf(pv.y, c[m + 1], acc[e]);

@@ -95,7 +95,7 @@ __device__ __forceinline__ int ranked_rows(const int *rank, int h, int r) {
 // Steps shared by both window-update kernels, for one head whose state is in
 // registers: apply the n staged tokens in order, scale, round to the storage
 // type, store the state once, and refresh the sketch from the same registers.
-template <int KIND, int DK, typename ST, int NC, bool READ>
+template <int KIND, int DK, typename ST, int NC, bool READ, bool SEQS>
 __device__ __forceinline__ void apply_store_refresh(float (&s)[NC][DK / 8], const float *sk, const float *su,
                                                     const float *sv, const float *sg, const float *sut,
                                                     const float *ss2, const float *sq, ST *__restrict__ S,
@@ -105,7 +105,7 @@ __device__ __forceinline__ void apply_store_refresh(float (&s)[NC][DK / 8], cons
     constexpr int EPL = TL::EPL;
     const int cl = NC == 8 ? l : l >> 1;  // the column whose reduced values this lane holds
     // the buffered tokens, in order
-    for (int t = 0; t < n; ++t) {
+    auto token = [&](int t) {
         float kv[EPL];
         lane_channels_smem<DK, ST>(sk + t * DK, l, kv);
         if (KIND == MAMBA2) {
@@ -117,22 +117,49 @@ __device__ __forceinline__ void apply_store_refresh(float (&s)[NC][DK / 8], cons
             }
 #pragma unroll
             for (int cc = 0; cc < NC; ++cc) axpy<EPL>(s[cc], kv, vv[cc]);
+        } else if constexpr (NC == 4) {
+            // two independent column pairs, each reduced over the octet on its own (lanes
+            // l < 4 end with the pair's first column, l >= 4 with its second), so that one
+            // pair's shuffles overlap the other pair's FMAs, and, with two tokens unrolled,
+            // the next token's dots
+            const bool hi = lane & 4;
+            float x[2];
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                const float d0 = dot<EPL>(kv, s[2 * p]), d1 = dot<EPL>(kv, s[2 * p + 1]);
+                float y = (hi ? d1 : d0) + __shfl_xor_sync(FULL, hi ? d0 : d1, 4);
+                y += __shfl_xor_sync(FULL, y, 2);
+                x[p] = y + __shfl_xor_sync(FULL, y, 1);
+            }
+            const float b2 = KIND == GDN ? ss2[t] : 1.f;
+            const float uA = sv[t * dv + c0 + hi] - b2 * x[0];
+            const float uB = sv[t * dv + c0 + 2 + hi] - b2 * x[1];
+            float uu[4] = {__shfl_sync(FULL, uA, 0, 8), __shfl_sync(FULL, uA, 4, 8),
+                           __shfl_sync(FULL, uB, 0, 8), __shfl_sync(FULL, uB, 4, 8)};
+            if (KIND == KDA) lane_channels_smem<DK, ST>(su + t * DK, l, kv);
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) axpy<EPL>(s[cc], kv, uu[cc]);
         } else {
             float d[NC];
 #pragma unroll
             for (int cc = 0; cc < NC; ++cc) d[cc] = dot<EPL>(kv, s[cc]);
-            float dsum;
-            if constexpr (NC == 8) dsum = octet_reduce_scatter(d, lane);
-            else dsum = octet_reduce4(d, lane);
+            const float dsum = octet_reduce_scatter(d, lane);
             const float vc = sv[t * dv + c0 + cl];
             const float u = KIND == GDN ? vc - ss2[t] * dsum : vc - dsum;
             float uu[NC];
-            if constexpr (NC == 8) octet_all_gather(u, uu);
-            else octet_all_gather4(u, uu);
+            octet_all_gather(u, uu);
             if (KIND == KDA) lane_channels_smem<DK, ST>(su + t * DK, l, kv);
 #pragma unroll
             for (int cc = 0; cc < NC; ++cc) axpy<EPL>(s[cc], kv, uu[cc]);
         }
+    };
+    // (two tokens per iteration only where the registers allow it without spilling: the
+    // plain update of dk = 128 heads)
+    if constexpr (KIND != MAMBA2 && NC == 4 && DK == 128 && !READ && !SEQS) {
+#pragma unroll 2
+        for (int t = 0; t < n; ++t) token(t);
+    } else {
+        for (int t = 0; t < n; ++t) token(t);
     }
 
     // final scale
@@ -295,7 +322,7 @@ update_window_kernel(ST *__restrict__ S, float *__restrict__ P, const float *__r
     }
     __syncthreads();
 
-    apply_store_refresh<KIND, DK, ST, NC, READ>(s, sk, su, sv, sg, sut, ss2, sq, S, P, o, head, dv, r, r, n,
+    apply_store_refresh<KIND, DK, ST, NC, READ, SEQS>(s, sk, su, sv, sg, sut, ss2, sq, S, P, o, head, dv, r, r, n,
                                           c0, l, lane);
 }
 
@@ -531,7 +558,7 @@ update_window_persistent(ST *__restrict__ S, float *__restrict__ P, const float 
         if (tid == 0 && w + ns < w_end) issue(w + ns, stage);
 
         if (!SEQS || head >= 0)  // CTA-uniform
-            apply_store_refresh<KIND, DK, ST, NC, READ>(s, sk, su, sv, sg, sut, ss2, sq, S, P, o, head, dv, r,
+            apply_store_refresh<KIND, DK, ST, NC, READ, SEQS>(s, sk, su, sv, sg, sut, ss2, sq, S, P, o, head, dv, r,
                                                         RANKED ? ranked_rows(rank, h, r) : r, n, c0, l,
                                                         lane);
     }

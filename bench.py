@@ -53,11 +53,16 @@ def parse():
     ap.add_argument("--state-dtype", choices=["f32", "bf16"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--cpu-seconds", type=float, default=16.0)
     ap.add_argument("--rank-avg", type=int, default=0,
                     help="also time the sketch path with a rank per head: this average, the config's r the largest")
     ap.add_argument("--stagger-share", default="2,2",
                     help="CTAs per SM for the decode and update kernels of the staggered schedule")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other workloads (GDN, KDA r = 4, 8, 16) of the single-GPU line")
+    ap.add_argument("--workload-steps", type=int, default=30)
+    ap.add_argument("--no-sweep", action="store_true", help="skip the GDN sweep of the single-GPU line")
+    ap.add_argument("--sweep-steps", type=int, default=10)
     return ap.parse_args()
 
 
@@ -250,24 +255,61 @@ class OracleSample:
                            bf16_state=self.cfg.state_dtype == "bf16")
         return (self.chunk / self.cfg.H) * self.cfg.W  # token-steps done
 
+    def step_full(self):
+        """The oracle's full-read path on the same sample: every token updates and reads the state."""
+        import oracle
+
+        oracle.fullread_path(self.cfg.kind, self.S0, self.ft, bf16_state=self.cfg.state_dtype == "bf16")
+        return (self.chunk / self.cfg.H) * self.cfg.W
+
     def describe(self, n_steps, seconds):
         return (f"{n_steps} x (oracle sketch path, fp64: sketch refresh, {self.cfg.W} sketch reads, window "
                 f"update) on {self.chunk} heads ({self.chunk / self.cfg.H:.2f} sequences x {self.cfg.H} heads) "
                 f"of the workload, {seconds:.1f} s")
 
 
-def cpu_oracle_rate(cfg, seconds: float):
-    """Oracle token-steps/s over repeated sample steps until `seconds` have passed."""
-    smp = OracleSample(cfg)
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+
+    return platform.processor() or "unknown"
+
+
+def _rate(fn, seconds: float):
     done, n = 0.0, 0
     t0 = time.perf_counter()
     while True:
-        done += smp.step()
+        done += fn()
         n += 1
         el = time.perf_counter() - t0
         if el >= seconds:
-            break
-    return done / el, smp.describe(n, el), smp.threads
+            return done / el, n, el
+
+
+def cpu_oracle_rate(cfg, seconds: float):
+    """The fp64 oracle on the host: its sketch path on all OpenMP threads (the reported value), its
+    full-read path on the same sample, and the sketch path on one thread.  About half of `seconds`
+    goes to the first, a quarter to each of the others."""
+    import oracle
+
+    smp = OracleSample(cfg)
+    rate, n, el = _rate(smp.step, 0.5 * seconds)
+    full, nf, elf = _rate(smp.step_full, 0.25 * seconds)
+    oracle.set_num_threads(1)
+    try:
+        one, n1, el1 = _rate(smp.step, 0.25 * seconds)
+    finally:
+        oracle.set_num_threads(smp.threads)
+    desc = (smp.describe(n, el) + f"; full-read path: {nf} x the same sample's {cfg.W} exact steps, {elf:.1f} s; "
+            f"one thread: {n1} sketch-path steps, {el1:.1f} s")
+    return {"value": rate, "unit": UNIT, "cores": smp.threads, "kind": "oracle", "sample": desc,
+            "fullread_value": full, "single_thread_value": one, "cpu_model": cpu_model()}
 
 
 def run_reference(args):
@@ -314,6 +356,305 @@ def reduce_max(x: float, device=None) -> float:
 def whole_job_rate(units_per_rank: float, world: int, t_max: float) -> float:
     """Replicas: every rank processes the same units; the job's rate is all units over the slowest rank."""
     return world * units_per_rank / t_max
+
+
+# ---------------------------------------------------------------- GPU arm: shared pieces
+def dims_of(cfg, B=None, r=None):
+    import recurrent_state_read_b200 as rs
+
+    return rs.dims(cfg.kind, cfg.B if B is None else B, cfg.H, cfg.dk, cfg.dv, cfg.r if r is None else r, cfg.W,
+                   cfg.torch_state_dtype, cfg.torch_qkv_dtype)
+
+
+def prefill_state(cfg, dev, B=None):
+    """The start state: cfg.prefill tokens through the library's window update, from S = 0."""
+    import torch
+
+    import workloads as wl
+    from recurrent_state_read_b200.decode import prefill
+
+    B = cfg.B if B is None else B
+    d = dims_of(cfg, B=B)
+    S0 = torch.zeros(B, cfg.H, cfg.dv, cfg.dk, dtype=cfg.torch_state_dtype, device=dev)
+    P = torch.empty(B, cfg.H, cfg.dv, cfg.r, device=dev)
+    U0 = torch.zeros(cfg.H, cfg.r, cfg.dk, device=dev)
+    prefill(d, S0, P, U0, lambda t0, n: wl.token_block(cfg, "prefill", t0, n, device=dev, B=B), cfg.prefill)
+    return S0
+
+
+def calibration_states(cfg, dev):
+    """Final prefill states of the cfg.n_cal_seq calibration sequences (the "cal" token stream)."""
+    import torch
+
+    import workloads as wl
+    from recurrent_state_read_b200.decode import prefill
+
+    dc = dims_of(cfg, B=cfg.n_cal_seq)
+    S_cal = torch.zeros(cfg.n_cal_seq, cfg.H, cfg.dv, cfg.dk, dtype=cfg.torch_state_dtype, device=dev)
+    P = torch.empty(cfg.n_cal_seq, cfg.H, cfg.dv, cfg.r, device=dev)
+    U0 = torch.zeros(cfg.H, cfg.r, cfg.dk, device=dev)
+    prefill(dc, S_cal, P, U0, lambda t0, n: wl.token_block(cfg, "cal", t0, n, device=dev), cfg.prefill)
+    return S_cal
+
+
+def calibrate(cfg, S_cal, q_cal, dev, r=None):
+    """Basis rows U and coefficient map R [H, r, dk] from the library's offline calibration."""
+    import torch
+
+    import recurrent_state_read_b200 as rs
+
+    r = cfg.r if r is None else r
+    dc = dims_of(cfg, B=cfg.n_cal_seq, r=r)
+    U = torch.empty(cfg.H, r, cfg.dk, device=dev)
+    R = torch.empty(cfg.H, r, cfg.dk, device=dev)
+    rs.sketchssm_calibrate_basis(dc, q_cal, S_cal, U, R)
+    return U, R
+
+
+def decode_windows(cfg, dev, B=None):
+    """NWIN distinct windows of decode tokens: window buffers and the time-major token planes."""
+    import workloads as wl
+    from recurrent_state_read_b200.decode import WindowBuffer
+
+    B = cfg.B if B is None else B
+    d = dims_of(cfg, B=B)
+    bufs, toks = [], []
+    for i in range(NWIN):
+        tok = wl.token_block(cfg, "decode", i * cfg.W, cfg.W, device=dev, B=B, with_query=True)
+        tok = {k: (None if v is None else v.contiguous()) for k, v in tok.items()}
+        b = WindowBuffer.empty(d, device=dev)
+        b.fill(tok)
+        bufs.append(b)
+        toks.append(tok)
+    return bufs, toks
+
+
+def capture_graph(fn, stream):
+    """fn's launches as a CUDA graph (one eager call first, outside capture, warms the launch path)."""
+    import torch
+
+    g = torch.cuda.CUDAGraph()
+    fn()
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    return g
+
+
+def timed_windows(parts, steps, warmup, stream, clocks, barrier):
+    """Replay, per step i, the graphs parts[0][i % NWIN], parts[1][i % NWIN], ... in order, with CUDA
+    events on the launching stream around each.  Returns (seconds over all steps, [seconds per part])."""
+    import torch
+
+    for i in range(warmup):
+        for p in parts:
+            p[i % NWIN].replay()
+    barrier()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)] for _ in range(steps)]
+    clocks.mark(True)
+    for i in range(steps):
+        evs[i][0].record(stream)
+        for k, p in enumerate(parts):
+            p[i % NWIN].replay()
+            evs[i][k + 1].record(stream)
+    barrier()
+    clocks.mark(False)
+    total = evs[0][0].elapsed_time(evs[-1][-1]) / 1e3
+    per = [sum(e[k].elapsed_time(e[k + 1]) for e in evs) / 1e3 for k in range(len(parts))]
+    return total, per
+
+
+def kernel_entry(bytes_, seconds, launches, peak):
+    ms = 1e3 * seconds / launches
+    gbps = bytes_ / ms / 1e6
+    return {"us_per_launch": 1e3 * ms, "algorithmic_bytes": bytes_, "GBps": gbps, "frac_of_peak": gbps / peak,
+            "nominal_8TBps_frac": gbps / 8000.0}
+
+
+def measured_gate(cfg, speedup):
+    """The speed target on measured DRAM bytes: the sketch path must beat the full-read path by at
+    least 0.8 x (full-read DRAM bytes / sketch DRAM bytes per token-step), both from one committed
+    ncu capture of each path's whole window (all kernels) whose kernel sources match these."""
+    p = os.path.join(ROOT, "profiles", f"traffic_gate_{cfg.kind}.txt")
+    if not os.path.exists(p):
+        return None
+    kv = {}
+    with open(p) as f:
+        for line in f:
+            if ":" in line and not line.startswith(" "):
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+    if (kv.get("csrc_sha256") or "").split()[:1] != [csrc_hash()] or kv.get("workload_key") != workload_key(cfg):
+        return None
+    try:
+        full = float(kv["fullread_dram_bytes_per_token_step"])
+        sk = float(kv["sketch_dram_bytes_per_token_step"])
+    except (KeyError, ValueError):
+        return None
+    ratio = full / sk
+    return {"fullread_dram_bytes_per_token_step": full, "sketch_dram_bytes_per_token_step": sk,
+            "measured_bytes_ratio": ratio, "bar": 0.8 * ratio, "speedup": speedup, "met": speedup >= 0.8 * ratio,
+            "source": os.path.relpath(p, ROOT)}
+
+
+def approx_error(d, S, P, U, R, buf, tok, dev):
+    """Relative L2 error of the sketch path's outputs against the exact read on one window."""
+    import torch
+
+    from recurrent_state_read_b200.decode import fullread_window, sketch_window
+
+    W = d.W
+    out = torch.empty(W, d.B, d.H, d.dv, device=dev)
+    out_f = torch.empty_like(out)
+    S_a, Sf_a, P_a = S.clone(), S.clone(), P.clone()
+    sketch_window(d, S_a, P_a, U, R, buf, out)
+    fullread_window(d, Sf_a, tok, out_f)
+    torch.cuda.synchronize()
+    return float(torch.linalg.vector_norm((out - out_f).double()) / torch.linalg.vector_norm(out_f.double()))
+
+
+def measure_workload(cfg, dev, stream, clocks, barrier, steps, warmup, peak):
+    """One workload's sketch path (decode steps + window update), full-read path and ReplaySSM-style
+    path, each over the same NWIN windows, with per-kernel rooflines, the traffic ratios and the
+    sketch's approximation error on the first window."""
+    import torch
+
+    import recurrent_state_read_b200 as rs
+    import workloads as wl
+    from recurrent_state_read_b200.decode import fullread_window
+
+    d = dims_of(cfg)
+    bm = bytes_model(cfg)
+    S0 = prefill_state(cfg, dev)
+    S_cal = calibration_states(cfg, dev)
+    U, R = calibrate(cfg, S_cal, wl.calibration_queries(cfg, device=dev), dev)
+    del S_cal
+    bufs, toks = decode_windows(cfg, dev)
+    W = cfg.W
+    S = S0.clone()
+    P = torch.empty(cfg.B, cfg.H, cfg.dv, cfg.r, device=dev)
+    rs.sketchssm_update_window(d, S, P, U, None, None, None, None, 0)
+    approx = approx_error(d, S, P, U, R, bufs[0], toks[0], dev)
+    out = torch.empty(W, cfg.B, cfg.H, cfg.dv, device=dev)
+    Sf, Sr = S0.clone(), S0.clone()
+    g_dec = [capture_graph(lambda b=b: [rs.sketchssm_decode_step(d, P, R, b.q[j - 1], b.k, b.v, b.alpha, b.beta, j,
+                                                                 out[j - 1]) for j in range(1, W + 1)], stream)
+             for b in bufs]
+    g_upd = [capture_graph(lambda b=b: rs.sketchssm_update_window(d, S, P, U, b.k, b.v, b.alpha, b.beta, W), stream)
+             for b in bufs]
+    g_full = [capture_graph(lambda t=t: fullread_window(d, Sf, t, out), stream) for t in toks]
+    g_rdec = [capture_graph(lambda b=b: [rs.sketchssm_replay_decode_step(d, Sr, b.q[j - 1], b.k, b.v, b.alpha,
+                                                                         b.beta, j, out[j - 1])
+                                         for j in range(1, W + 1)], stream) for b in bufs]
+    g_rupd = [capture_graph(lambda b=b: rs.sketchssm_update_window(d, Sr, None, None, b.k, b.v, b.alpha, b.beta, W),
+                            stream) for b in bufs]
+    t_s, (t_dec, t_upd) = timed_windows([g_dec, g_upd], steps, warmup, stream, clocks, barrier)
+    t_f, _ = timed_windows([g_full], steps, warmup, stream, clocks, barrier)
+    t_r, _ = timed_windows([g_rdec, g_rupd], steps, warmup, stream, clocks, barrier)
+    del g_dec, g_upd, g_full, g_rdec, g_rupd
+    tok_steps = steps * cfg.B * W
+    kernels = {"update_window": kernel_entry(bm["update"], t_upd, steps, peak),
+               "decode_step": kernel_entry(bm["decode_avg"], t_dec, steps * W, peak),
+               "fullread_decode": kernel_entry(bm["fullread"], t_f, steps * W, peak)}
+    dominant = "update_window" if t_upd >= t_dec else "decode_step"
+    value, value_f = tok_steps / t_s, tok_steps / t_f
+    speedup = value / value_f
+    state_ratio = (2 * W * bm["S"]) / (2 * bm["S"] + (W + 1) * bm["P"])
+    return {
+        "workload": config_json(cfg)["workload"], "value": value, "unit": UNIT, "steps": steps, "warmup": warmup,
+        "ms_per_step": 1e3 * t_s / steps, "kernels": kernels,
+        "roofline": {"bound": "hbm", "kernel": dominant, "achieved": kernels[dominant]["GBps"], "peak": peak,
+                     "unit": "GB/s", "frac": kernels[dominant]["frac_of_peak"],
+                     "nominal_8TBps_frac": kernels[dominant]["nominal_8TBps_frac"]},
+        "sketch_window_GBps": bm["sketch_step"] / (t_s / steps) / 1e9,
+        "fullread": {"value": value_f, "unit": UNIT, "ms_per_step": 1e3 * t_f / steps},
+        "replay": {"value": tok_steps / t_r, "unit": UNIT, "ms_per_step": 1e3 * t_r / steps},
+        "sketch_vs_fullread": {
+            "speedup": speedup,
+            "algorithmic_bytes_per_token_step": {"sketch": bm["sketch_step"] / (cfg.B * W),
+                                                 "fullread": bm["full_step"] / (cfg.B * W)},
+            "algorithmic_bytes_ratio": bm["full_step"] / bm["sketch_step"],
+            "state_bytes_ratio": state_ratio,
+            "gate_on_state_bytes": {"bar": 0.8 * state_ratio, "met": speedup >= 0.8 * state_ratio},
+            "gate_on_measured_bytes": measured_gate(cfg, speedup),
+            "approx_rel_l2_first_window": approx},
+    }
+
+
+SWEEP_B = (64, 256, 1024)
+SWEEP_R = (4, 8, 16, 32)
+SWEEP_W = (4, 8, 16, 32)
+SWEEP_DT = ("f32", "bf16")
+
+
+def run_sweep(dev, stream, clocks, barrier, steps, warmup, peak):
+    """The GDN sweep on the sketch path: B x r x W x state dtype (96 points), and the full-read path
+    per (B, state dtype).  Per (W, dtype) the calibration states are prefilled once and calibrated
+    at each r; per (B, W, dtype) the start state is prefilled once and timed at each r."""
+    import torch
+
+    import recurrent_state_read_b200 as rs
+    import workloads as wl
+    from recurrent_state_read_b200.decode import fullread_window
+
+    points, fulls = [], []
+    for sdt in SWEEP_DT:
+        for W in SWEEP_W:
+            base = wl.workload(4, W=W, state_dtype=sdt)
+            S_cal = calibration_states(base, dev)
+            q_cal = wl.calibration_queries(base, device=dev)
+            bases = {r: calibrate(base, S_cal, q_cal, dev, r=r) for r in SWEEP_R}
+            del S_cal
+            for B in SWEEP_B:
+                cfgB = wl.workload(4, B=B, W=W, state_dtype=sdt)
+                S0 = prefill_state(cfgB, dev)
+                bufs, toks = decode_windows(cfgB, dev)
+                out = torch.empty(W, B, cfgB.H, cfgB.dv, device=dev)
+                for r in SWEEP_R:
+                    cfg = wl.workload(4, B=B, W=W, r=r, state_dtype=sdt)
+                    d = dims_of(cfg)
+                    bm = bytes_model(cfg)
+                    U, R = bases[r]
+                    S = S0.clone()
+                    P = torch.empty(B, cfg.H, cfg.dv, r, device=dev)
+                    rs.sketchssm_update_window(d, S, P, U, None, None, None, None, 0)
+                    g_dec = [capture_graph(lambda b=b: [rs.sketchssm_decode_step(d, P, R, b.q[j - 1], b.k, b.v,
+                                                                                 b.alpha, b.beta, j, out[j - 1])
+                                                        for j in range(1, W + 1)], stream) for b in bufs]
+                    g_upd = [capture_graph(lambda b=b: rs.sketchssm_update_window(d, S, P, U, b.k, b.v, b.alpha,
+                                                                                  b.beta, W), stream) for b in bufs]
+                    t_s, (t_dec, t_upd) = timed_windows([g_dec, g_upd], steps, warmup, stream, clocks, barrier)
+                    del g_dec, g_upd, S, P
+                    upd = kernel_entry(bm["update"], t_upd, steps, peak)
+                    dec = kernel_entry(bm["decode_avg"], t_dec, steps * W, peak)
+                    win_gbps = bm["sketch_step"] / (t_s / steps) / 1e9
+                    points.append({
+                        "B": B, "r": r, "W": W, "state": sdt, "value": steps * B * W / t_s,
+                        "ms_per_step": 1e3 * t_s / steps,
+                        "bytes_per_token_step": bm["sketch_step"] / (B * W),
+                        "window_GBps": win_gbps, "window_frac": win_gbps / peak,
+                        "update_us": upd["us_per_launch"], "update_GBps": upd["GBps"], "update_frac": upd["frac_of_peak"],
+                        "decode_us": dec["us_per_launch"], "decode_GBps": dec["GBps"], "decode_frac": dec["frac_of_peak"]})
+                if W == 16:  # the full-read path does not depend on W or r
+                    d = dims_of(cfgB)
+                    bm = bytes_model(cfgB)
+                    Sf = S0.clone()
+                    g_full = [capture_graph(lambda t=t: fullread_window(d, Sf, t, out), stream) for t in toks]
+                    t_f, _ = timed_windows([g_full], steps, warmup, stream, clocks, barrier)
+                    del g_full, Sf
+                    fk = kernel_entry(bm["fullread"], t_f, steps * W, peak)
+                    fulls.append({"B": B, "state": sdt, "value": steps * B * W / t_f,
+                                  "bytes_per_token_step": bm["full_step"] / (B * W),
+                                  "us_per_step": fk["us_per_launch"], "GBps": fk["GBps"], "frac": fk["frac_of_peak"]})
+                del S0, bufs, toks, out
+                torch.cuda.empty_cache()
+    for p in points:  # speed-up over the full-read path of the same batch and state dtype
+        f = next(x for x in fulls if x["B"] == p["B"] and x["state"] == p["state"])
+        p["speedup_vs_fullread"] = p["value"] / f["value"]
+    return {"workload": "GDN sweep: H=32 dk=dv=128, q/k/v bf16; B x r x W x state dtype",
+            "axes": {"B": list(SWEEP_B), "r": list(SWEEP_R), "W": list(SWEEP_W), "state": list(SWEEP_DT)},
+            "steps_per_point": steps, "warmup_per_point": warmup, "unit": UNIT, "peak_GBps": peak,
+            "points": points, "fullread": fulls}
 
 
 # ---------------------------------------------------------------- GPU arm
@@ -689,15 +1030,32 @@ def run_ours(args):
         t_e2e = max_over_ranks(ee0.elapsed_time(ee1) / 1e3)
         e2e = {"value": whole_job_rate(args.steps * cfg.B * cfg.W, world, t_e2e), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": 1e3 * t_e2e / args.steps,
+               "pcie_GBps": (h2d + d2h) / (t_e2e / args.steps) / 1e9,
                "path": "python binding -> C ABI; every window's inputs copied in from pinned host memory and "
                        "its outputs copied out, inside the timed region, overlapped with the neighbouring "
-                       "windows' compute on two copy streams"}
+                       "windows' compute on two copy streams (bound by the host link, not the kernels)"}
+        del g_dec_e
+    peak, peak_src = hbm_peak()
+
+    # the other workloads and the GDN sweep (single GPU only; the scaling runs time the headline)
+    extra = {}
+    if world == 1 and not args.no_workloads:
+        del g_st
+        g_st = None
+        torch.cuda.empty_cache()
+        extra["workloads"] = {}
+        for name, wcfg in (("gdn", wl.workload(2)), ("kda_r4", wl.workload(3, r=4)), ("kda_r8", wl.workload(3, r=8)),
+                           ("kda_r16", wl.workload(3, r=16))):
+            extra["workloads"][name] = measure_workload(wcfg, dev, stream, clocks, barrier, args.workload_steps, 3, peak)
+            torch.cuda.empty_cache()
+    if world == 1 and not args.no_sweep:
+        extra["sweep"] = run_sweep(dev, stream, clocks, barrier, args.sweep_steps, 3, peak)
+        torch.cuda.empty_cache()
     clk = clocks.stop()
 
     tok_per_step = cfg.B * cfg.W
     value = whole_job_rate(args.steps * tok_per_step, world, t_sketch)
     value_full = whole_job_rate(args.steps * tok_per_step, world, t_full)
-    peak, peak_src = hbm_peak()
     upd_ms = 1e3 * t_upd / args.steps
     dec_ms = 1e3 * t_dec / (args.steps * cfg.W)
     full_ms = 1e3 * t_full / (args.steps * cfg.W)
@@ -711,6 +1069,8 @@ def run_ours(args):
     }
     for k in kernels.values():
         k["frac_of_peak"] = k["GBps"] / peak
+        k["nominal_8TBps_frac"] = k["GBps"] / 8000.0
+    state_ratio = (2 * cfg.W * bm["S"]) / (2 * bm["S"] + (cfg.W + 1) * bm["P"])
     dominant = "update_window" if t_upd >= t_dec else "decode_step"
     kd = kernels[dominant]
     traffic = profiled_traffic(f"{dominant}_{cfg.kind}", cfg)
@@ -762,7 +1122,9 @@ def run_ours(args):
             "algorithmic_bytes_per_token_step": {"sketch": bm["sketch_step"] / tok_per_step,
                                                  "fullread": bm["full_step"] / tok_per_step},
             "algorithmic_bytes_ratio": bm["full_step"] / bm["sketch_step"],
-            "state_bytes_ratio": (2 * cfg.W * bm["S"]) / (2 * bm["S"] + (cfg.W + 1) * bm["P"]),
+            "state_bytes_ratio": state_ratio,
+            "gate_on_state_bytes": {"bar": 0.8 * state_ratio, "met": value / value_full >= 0.8 * state_ratio},
+            "gate_on_measured_bytes": measured_gate(cfg, value / value_full),
             "approx_rel_l2_first_window": approx,
         },
         "gpu_launches": args.steps * (cfg.W + 1),
@@ -770,9 +1132,9 @@ def run_ours(args):
     }
     if e2e is not None:
         line["e2e"] = e2e
+    line.update(extra)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, desc, cores = cpu_oracle_rate(cfg, args.cpu_seconds)
-        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+        line["cpu_baseline"] = cpu_oracle_rate(cfg, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
     del g_dec, g_upd, g_full, g_x, g_rdec, g_rupd, g_st, g_wy

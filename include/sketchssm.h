@@ -99,6 +99,9 @@ int sketchssm_version(void);
  * For every head: apply buffered tokens t = 0 .. n_tokens-1 of the window
  * buffer to S, in order, exactly (fp32 arithmetic); store S (rounded to
  * state_dtype, nearest-even, for SKSSM_BF16); then write P = S_stored^T U.
+ * Any decay values are accepted, including 0 (a state reset) and windows whose
+ * decay product underflows or exceeds the fp32 range: such a head is updated
+ * token by token instead of through the running decay scale.
  * n_tokens = 0 is a sketch refresh only (S is read, not written).
  *   S        in/out [B][H][dv][dk] state_dtype
  *   P        out    [B][H][dv][r] fp32; NULL: no sketch refresh (a plain buffered

@@ -62,8 +62,9 @@ def _load():
         lib.orc_update_window.argtypes = [i, i, i, i, i, i, P, P, P, P, P, P, P, i]
         lib.orc_sketch_read.argtypes = [i, i, i, i, i, i, P, P, P, P, P, P, P, P, P, P]
         lib.orc_round_bf16.argtypes = [ctypes.c_size_t, P]
+        lib.orc_set_num_threads.argtypes = [i]
         for f in ("orc_exact_steps", "orc_read", "orc_update_window", "orc_sketch_read",
-                  "orc_round_bf16", "orc_num_threads"):
+                  "orc_round_bf16", "orc_num_threads", "orc_set_num_threads"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -71,6 +72,11 @@ def _load():
 
 def num_threads() -> int:
     return int(_load().orc_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """OpenMP threads of the following oracle calls (timing only; results do not depend on it)."""
+    _check(_load().orc_set_num_threads(int(n)), "set_num_threads")
 
 
 def f64(x) -> np.ndarray:

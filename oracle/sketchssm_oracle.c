@@ -112,6 +112,17 @@ int orc_num_threads(void)
 #endif
 }
 
+/* Threads the following calls use (n >= 1); a timing control only, no effect on results:
+ * every head is computed by one thread, in the same order, whatever the count. */
+int orc_set_num_threads(int n)
+{
+    if (n < 1) return -1;
+#ifdef _OPENMP
+    omp_set_num_threads(n);
+#endif
+    return 0;
+}
+
 /* Per-step exact recurrence over T tokens for N heads (the full-read path):
  * for t = 0..T-1: S <- token t; if Q: O[t] = S^T Q[t].  With bf16_state the
  * state is rounded to bf16 after every token (after that token's read, which

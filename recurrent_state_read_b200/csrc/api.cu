@@ -8,11 +8,7 @@
 
 using namespace skssm;
 
-namespace {
-
-bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
-
-int check_dims(const sketchssm_dims *d) {
+int skssm::check_dims(const sketchssm_dims *d) {
     if (!d) return SKSSM_ERR_NULL;
     if (d->kind < SKSSM_MAMBA2 || d->kind > SKSSM_KDA) return SKSSM_ERR_DIMS;
     if (d->state_dtype != SKSSM_F32 && d->state_dtype != SKSSM_BF16) return SKSSM_ERR_DTYPE;
@@ -25,6 +21,10 @@ int check_dims(const sketchssm_dims *d) {
     if ((int64_t)d->B * d->H >= (int64_t)1 << 31) return SKSSM_ERR_DIMS;
     return SKSSM_OK;
 }
+
+namespace {
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 // window buffer / token pointers: k, v 16 B; alpha, beta 4 B
 int check_tokens(const sketchssm_dims *d, const void *k, const void *v, const float *alpha,

@@ -318,38 +318,11 @@ static size_t basis_smem() {
 
 int launch_calibrate(const sketchssm_dims &d, const float *q_cal, int Nq, const void *S_cal, int Ns,
                      double ridge, float *U, float *R, void *workspace, cudaStream_t stream, double *lam) {
-    double *G = static_cast<double *>(workspace);
-    double *C = G + (size_t)d.H * d.dk * d.dk;
-    double *T = C + (size_t)d.H * d.dk * d.dk;
-    auto run = [&](auto DKc) -> int {
-        constexpr int DK = decltype(DKc)::value;
-        const dim3 ggrid((DK / 32) * (DK / 32), d.H);
-        // G from the states: row (s, c) of head h at S_cal + ((s*H + h)*dv + c)*DK
-        const size_t sh = (size_t)d.dv * DK, sb = (size_t)d.H * d.dv * DK;
-        if (d.state_dtype == SKSSM_F32)
-            gram_kernel<float, DK><<<ggrid, 256, 0, stream>>>(static_cast<const float *>(S_cal), sh, sb,
-                                                              d.dv, Ns * d.dv, 1.0 / Ns, G);
-        else
-            gram_kernel<__nv_bfloat16, DK><<<ggrid, 256, 0, stream>>>(
-                static_cast<const __nv_bfloat16 *>(S_cal), sh, sb, d.dv, Ns * d.dv, 1.0 / Ns, G);
-        if (launch_status() != SKSSM_OK) return SKSSM_ERR_CUDA;
-        // C from the queries: row n of head h at q_cal + (h*Nq + n)*DK
-        gram_kernel<float, DK><<<ggrid, 256, 0, stream>>>(q_cal, (size_t)Nq * DK, 0, Nq, Nq, 1.0 / Nq, C);
-        if (launch_status() != SKSSM_OK) return SKSSM_ERR_CUDA;
-        const size_t smem = basis_smem<DK>();
-        if (cudaFuncSetAttribute(basis_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem) != cudaSuccess)
-            return SKSSM_ERR_CUDA;
-        basis_kernel<DK><<<d.H, BASIS_THREADS, smem, stream>>>(G, C, T, d.r, ridge, U, R, lam);
-        return launch_status();
-    };
-    if (d.dk == 64) return run(std::integral_constant<int, 64>());
-    if (d.dk == 128) return run(std::integral_constant<int, 128>());
-    return SKSSM_ERR_DIMS;
+    return launch_calibrate_heads(d, q_cal, Nq, S_cal, Ns, ridge, U, R, workspace, 0, d.H, stream, lam);
 }
 
-// Heads [h0, h0 + hc) only, with a workspace sized for hc heads: the same three
-// kernels as launch_calibrate, with every head-indexed pointer offset to h0.
+// Heads [h0, h0 + hc) only, with a workspace sized for hc heads: G and C (fp64 Gram
+// kernels), then the per-head basis, with every head-indexed pointer offset to h0.
 int launch_calibrate_heads(const sketchssm_dims &d, const float *q_cal, int Nq, const void *S_cal,
                            int Ns, double ridge, float *U, float *R, void *workspace, int h0, int hc,
                            cudaStream_t stream, double *lam) {

@@ -29,21 +29,10 @@ constexpr int MAX_DEVICES = 64;
 // refers to a host-side shadow.  The device address is looked up per device.
 static __device__ __align__(256) double g_calib_scratch[CALIB_SCRATCH_BYTES / sizeof(double)];
 
+// Device address of the scratch per device, looked up on first use.  A failed
+// lookup is not recorded, so the next call on that device tries again.
+std::mutex g_setup_mu;
 void *g_scratch_addr[MAX_DEVICES];
-cudaError_t g_setup_status[MAX_DEVICES];
-std::once_flag g_setup_once[MAX_DEVICES];
-
-int check(const sketchssm_dims *d) {
-    if (!d) return SKSSM_ERR_NULL;
-    if (d->kind < SKSSM_MAMBA2 || d->kind > SKSSM_KDA) return SKSSM_ERR_DIMS;
-    if (d->state_dtype != SKSSM_F32 && d->state_dtype != SKSSM_BF16) return SKSSM_ERR_DTYPE;
-    if (d->qkv_dtype != SKSSM_F32 && d->qkv_dtype != SKSSM_BF16) return SKSSM_ERR_DTYPE;
-    if (d->dk != 64 && d->dk != 128) return SKSSM_ERR_DIMS;
-    if (d->dv != 64 && d->dv != 128) return SKSSM_ERR_DIMS;
-    if (!((d->r >= 1 && d->r <= 32) || d->r == d->dk)) return SKSSM_ERR_DIMS;
-    if (d->W < 1 || d->W > 64 || d->B < 1 || d->H < 1) return SKSSM_ERR_DIMS;
-    return SKSSM_OK;
-}
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -52,7 +41,7 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 extern "C" int sketchssm_calibrate_basis_noalloc(const sketchssm_dims *d, const float *q_cal, int Nq,
                                                  const void *S_cal, int Ns, double ridge, float *U,
                                                  float *R, void *stream) {
-    int rc = check(d);
+    int rc = skssm::check_dims(d);
     if (rc) return rc;
     if (!q_cal || !S_cal || !U || !R) return SKSSM_ERR_NULL;
     if (Nq < 1 || Ns < 1 || !(ridge >= 0.0)) return SKSSM_ERR_RANGE;
@@ -66,14 +55,20 @@ extern "C" int sketchssm_calibrate_basis_noalloc(const sketchssm_dims *d, const 
     // Set-up, once per device, with that device current: the scratch's device address.
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return SKSSM_ERR_CUDA;
-    std::call_once(g_setup_once[dev], [dev] {
-        g_setup_status[dev] = cudaGetSymbolAddress(&g_scratch_addr[dev], g_calib_scratch);
-    });
-    if (g_setup_status[dev] != cudaSuccess || !g_scratch_addr[dev]) return SKSSM_ERR_CUDA;
+    void *scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_setup_mu);
+        if (!g_scratch_addr[dev]) {
+            void *p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_calib_scratch) != cudaSuccess || !p) return SKSSM_ERR_CUDA;
+            g_scratch_addr[dev] = p;
+        }
+        scratch = g_scratch_addr[dev];
+    }
 
     for (int h0 = 0; h0 < d->H; h0 += heads_per_pass) {
         const int hc = d->H - h0 < heads_per_pass ? d->H - h0 : heads_per_pass;
-        rc = skssm::launch_calibrate_heads(*d, q_cal, Nq, S_cal, Ns, ridge, U, R, g_scratch_addr[dev], h0,
+        rc = skssm::launch_calibrate_heads(*d, q_cal, Nq, S_cal, Ns, ridge, U, R, scratch, h0,
                                            hc, (cudaStream_t)stream);
         if (rc) return rc;
     }

@@ -559,13 +559,7 @@ int launch_decode_step(const sketchssm_dims &d, const float *P, const float *R, 
                 const size_t dsmem = (size_t)DEC_WARPS * DEC_DEEP_STAGES * DeepStage<KIND, DK, DV, QT>::bytes(8, j);
                 if (dsmem <= 227 * 1024) {
                     auto dk = decode_step_deep<KIND, DK, DV, QT, DEC_DEEP_STAGES>;
-                    static bool d_opted_in = false;
-                    if (!d_opted_in) {
-                        if (cudaFuncSetAttribute(dk, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-                            cudaSuccess)
-                            return SKSSM_ERR_CUDA;
-                        d_opted_in = true;
-                    }
+                    if (allow_max_smem(reinterpret_cast<const void *>(dk)) != SKSSM_OK) return SKSSM_ERR_CUDA;
                     int sms = 0, per_sm = 0;
                     if (sm_count(&sms) != SKSSM_OK ||
                         blocks_per_sm(reinterpret_cast<const void *>(dk), DEC_WARPS * 32, dsmem, &per_sm) != SKSSM_OK)
@@ -588,13 +582,7 @@ int launch_decode_step(const sketchssm_dims &d, const float *P, const float *R, 
                     auto persist = [&](auto JVc, auto RANKEDc) -> int {
                         auto pk = decode_step_persistent<KIND, DK, DV, QT, decltype(JVc)::value,
                                                          decltype(RANKEDc)::value>;
-                        static bool p_opted_in = false;
-                        if (!p_opted_in) {
-                            if (cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-                                cudaSuccess)
-                                return SKSSM_ERR_CUDA;
-                            p_opted_in = true;
-                        }
+                        if (allow_max_smem(reinterpret_cast<const void *>(pk)) != SKSSM_OK) return SKSSM_ERR_CUDA;
                         int sms = 0, per_sm = 0;
                         if (sm_count(&sms) != SKSSM_OK ||
                             blocks_per_sm(reinterpret_cast<const void *>(pk), DEC_WARPS * 32, psmem, &per_sm) !=
@@ -621,13 +609,7 @@ int launch_decode_step(const sketchssm_dims &d, const float *P, const float *R, 
             const int jc = j < jmax ? j : jmax;
             const size_t smem = (size_t)DEC_WARPS * DecSlots<KIND, DK, DV, QT>::bytes(jc);
             auto kern = decode_step_kernel<KIND, DK, DV, QT>;
-            static bool opted_in = false;
-            if (!opted_in) {
-                if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-                    cudaSuccess)
-                    return SKSSM_ERR_CUDA;
-                opted_in = true;
-            }
+            if (allow_max_smem(reinterpret_cast<const void *>(kern)) != SKSSM_OK) return SKSSM_ERR_CUDA;
             kern<<<grid, DEC_WARPS * 32, smem, stream>>>(P, R, static_cast<const QT *>(q),
                                                          static_cast<const QT *>(k), static_cast<const QT *>(v),
                                                          alpha, beta, o, d.B, d.H, d.r, j, d.W, jc, jv);

@@ -4,11 +4,16 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <mutex>
 #include <type_traits>
+#include <vector>
 
 #include "sketchssm.h"
 
 namespace skssm {
+
+// Validation of a dims struct shared by every entry point: SKSSM_OK or the status to return.
+int check_dims(const sketchssm_dims *d);
 
 // Call fn(kind, dk, state type, qkv type) with compile-time constants for the
 // supported combinations; returns SKSSM_ERR_DIMS / SKSSM_ERR_DTYPE otherwise.
@@ -49,26 +54,47 @@ int launch_update_window(const sketchssm_dims &d, void *S, float *P, const float
 int update_wait_giveups(bool reset, unsigned *count);
 int decode_wait_giveups(bool reset, unsigned *count);
 
+// Opt a kernel into the largest dynamic shared memory (227 KB) on the current device.  The
+// attribute belongs to the kernel's module in each device context, so it is set once per
+// (kernel, device); the record is guarded for calls from several host threads, and a failed
+// attempt is not recorded (the next launch tries again).
+inline int allow_max_smem(const void *kern) {
+    constexpr int MAX_SMEM = 227 * 1024;
+    static std::mutex mu;
+    static std::vector<std::pair<const void *, int>> done;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SKSSM_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    for (const auto &e : done)
+        if (e.first == kern && e.second == dev) return SKSSM_OK;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, MAX_SMEM) != cudaSuccess)
+        return SKSSM_ERR_CUDA;
+    done.emplace_back(kern, dev);
+    return SKSSM_OK;
+}
+
 // Resident CTAs per SM of a kernel at this block size and dynamic shared memory.
 // The occupancy query costs host time comparable to a short kernel, so results are
 // cached per calling thread (a few entries, replaced round-robin).
 inline int blocks_per_sm(const void *kern, int threads, size_t smem, int *per_sm) {
     struct Entry {
         const void *fn;
-        int threads;
+        int dev, threads;
         size_t smem;
         int per;
     };
     thread_local Entry cache[8] = {};
     thread_local int next = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SKSSM_ERR_CUDA;
     for (const Entry &e : cache)
-        if (e.fn == kern && e.threads == threads && e.smem == smem) {
+        if (e.fn == kern && e.dev == dev && e.threads == threads && e.smem == smem) {
             *per_sm = e.per;
             return SKSSM_OK;
         }
     int per = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, kern, threads, smem) != cudaSuccess) return SKSSM_ERR_CUDA;
-    cache[next] = Entry{kern, threads, smem, per};
+    cache[next] = Entry{kern, dev, threads, smem, per};
     next = (next + 1) & 7;
     *per_sm = per;
     return SKSSM_OK;

@@ -105,13 +105,7 @@ int launch_replay_decode(const sketchssm_dims &d, const void *S, const void *q, 
             using SL = DecSlots<KIND, DK, DV, QT>;
             const size_t smem = 16 + (size_t)j * (SL::KB + SL::VB + SL::AB) + (DK + DV) * sizeof(float);
             auto kern = replay_decode_kernel<KIND, DK, DV, ST, QT>;
-            static bool opted_in = false;
-            if (!opted_in) {
-                if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-                    cudaSuccess)
-                    return SKSSM_ERR_CUDA;
-                opted_in = true;
-            }
+            if (allow_max_smem(reinterpret_cast<const void *>(kern)) != SKSSM_OK) return SKSSM_ERR_CUDA;
             kern<<<NH, DV, smem, stream>>>(static_cast<const ST *>(S), static_cast<const QT *>(q),
                                            static_cast<const QT *>(k), static_cast<const QT *>(v), alpha, beta, o,
                                            j, d.W);

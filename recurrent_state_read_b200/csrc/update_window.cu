@@ -22,12 +22,29 @@
 // KDA folds its per-channel decay the same way with g_{t,i} = prod a_{s,i}:
 //   d = (k (.) g_t) . S^;  S^ += (b_t k / g_t) (v - d)
 // and the stored state is S = g (.) S^ (scalar g for Mamba-2 and GDN).
+//
+// The fold divides by g_t, so it holds only while every running product stays
+// a normal fp32 number: a zero decay (a state reset), or a window whose decay
+// product underflows (16 tokens at a = 1e-3, a KDA channel decaying at 1e-6),
+// would turn 1/g_t into inf and the state into 0 * inf = NaN.  Each head checks
+// its products first; if any g_t (any channel's, for KDA) leaves
+// [FOLD_LO, FOLD_HI] or is not finite, that head takes the plain recurrence
+// instead -- per token the state is multiplied by the token's decay, then the
+// delta step runs with g = 1 -- which divides by nothing.  The decision is
+// per head and uniform over the CTA; workload decays (a ~ 0.9) never leave
+// the range, so the fast path is what runs there.
 #include "internal.h"
 #include "state_tile.cuh"
 
 namespace skssm {
 
 constexpr int UPD_NC = 8;  // value columns per lane (state_tile.cuh)
+
+// Range of the running decay product g_t inside which the fold is used.  With
+// |g_t| >= 2^-64 the folded values stay below 2^64 |b v| per token, far from
+// fp32 overflow; a product outside the range (or NaN) selects the plain path.
+constexpr float FOLD_LO = 0x1p-64f, FOLD_HI = 0x1p64f;
+__device__ __forceinline__ bool fold_ok(float g) { return g >= FOLD_LO && g <= FOLD_HI; }
 
 // bounded waits that gave up, and sequence indices out of range, in either update kernel
 __device__ unsigned g_update_wait_giveups;
@@ -95,17 +112,41 @@ __device__ __forceinline__ int ranked_rows(const int *rank, int h, int r) {
 // Steps shared by both window-update kernels, for one head whose state is in
 // registers: apply the n staged tokens in order, scale, round to the storage
 // type, store the state once, and refresh the sketch from the same registers.
+//
+// Staged per token t (fast path, the fold):  sk = k (KDA: k (.) g_t);
+// sv = v b_t / g_t (GDN), v / g_t (Mamba-2), v (KDA); su = b_t k / g_t (KDA);
+// ss2 = b_t; sg = g_n (KDA: per channel).  Plain path (slow): sk = k;
+// sv = v b_t (GDN), v (Mamba-2, KDA); su = the decay row a_t (KDA); sa = a_t
+// (Mamba-2, GDN); ss2 = b_t; sg = 1.
 template <int KIND, int DK, typename ST, int NC, bool READ, bool SEQS>
 __device__ __forceinline__ void apply_store_refresh(float (&s)[NC][DK / 8], const float *sk, const float *su,
                                                     const float *sv, const float *sg, const float *sut,
-                                                    const float *ss2, const float *sq, ST *__restrict__ S,
-                                                    float *__restrict__ P, float *__restrict__ o, int head, int dv,
-                                                    int r, int r_used, int n, int c0, int l, int lane) {
+                                                    const float *ss2, const float *sa, const float *sq,
+                                                    ST *__restrict__ S, float *__restrict__ P,
+                                                    float *__restrict__ o, int head, int dv, int r, int r_used, int n,
+                                                    bool slow, int c0, int l, int lane) {
     using TL = TileLayout<DK, ST>;
     constexpr int EPL = TL::EPL;
     const int cl = NC == 8 ? l : l >> 1;  // the column whose reduced values this lane holds
     // the buffered tokens, in order
-    auto token = [&](int t) {
+    auto token = [&](int t, auto SLOWc) {
+        constexpr bool SLOW = decltype(SLOWc)::value;
+        if constexpr (SLOW) {  // the plain recurrence: the token's decay applied to the state itself
+            if constexpr (KIND == KDA) {
+                float av[EPL];
+                lane_channels_smem<DK, ST>(su + t * DK, l, av);
+#pragma unroll
+                for (int cc = 0; cc < NC; ++cc)
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) s[cc][e] *= av[e];
+            } else {
+                const float at = sa[t];
+#pragma unroll
+                for (int cc = 0; cc < NC; ++cc)
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) s[cc][e] *= at;
+            }
+        }
         float kv[EPL];
         lane_channels_smem<DK, ST>(sk + t * DK, l, kv);
         if (KIND == MAMBA2) {
@@ -132,11 +173,15 @@ __device__ __forceinline__ void apply_store_refresh(float (&s)[NC][DK / 8], cons
                 x[p] = y + __shfl_xor_sync(FULL, y, 1);
             }
             const float b2 = KIND == GDN ? ss2[t] : 1.f;
-            const float uA = sv[t * dv + c0 + hi] - b2 * x[0];
-            const float uB = sv[t * dv + c0 + 2 + hi] - b2 * x[1];
+            float uA = sv[t * dv + c0 + hi] - b2 * x[0];
+            float uB = sv[t * dv + c0 + 2 + hi] - b2 * x[1];
+            if constexpr (KIND == KDA && SLOW) {  // b_t (v - x): b is not folded into the keys
+                uA *= ss2[t];
+                uB *= ss2[t];
+            }
             float uu[4] = {__shfl_sync(FULL, uA, 0, 8), __shfl_sync(FULL, uA, 4, 8),
                            __shfl_sync(FULL, uB, 0, 8), __shfl_sync(FULL, uB, 4, 8)};
-            if (KIND == KDA) lane_channels_smem<DK, ST>(su + t * DK, l, kv);
+            if (KIND == KDA && !SLOW) lane_channels_smem<DK, ST>(su + t * DK, l, kv);
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) axpy<EPL>(s[cc], kv, uu[cc]);
         } else {
@@ -145,21 +190,25 @@ __device__ __forceinline__ void apply_store_refresh(float (&s)[NC][DK / 8], cons
             for (int cc = 0; cc < NC; ++cc) d[cc] = dot<EPL>(kv, s[cc]);
             const float dsum = octet_reduce_scatter(d, lane);
             const float vc = sv[t * dv + c0 + cl];
-            const float u = KIND == GDN ? vc - ss2[t] * dsum : vc - dsum;
+            float u = KIND == GDN ? vc - ss2[t] * dsum : vc - dsum;
+            if constexpr (KIND == KDA && SLOW) u *= ss2[t];
             float uu[NC];
             octet_all_gather(u, uu);
-            if (KIND == KDA) lane_channels_smem<DK, ST>(su + t * DK, l, kv);
+            if (KIND == KDA && !SLOW) lane_channels_smem<DK, ST>(su + t * DK, l, kv);
 #pragma unroll
             for (int cc = 0; cc < NC; ++cc) axpy<EPL>(s[cc], kv, uu[cc]);
         }
     };
-    // (two tokens per iteration only where the registers allow it without spilling: the
-    // plain update of dk = 128 heads)
-    if constexpr (KIND != MAMBA2 && NC == 4 && DK == 128 && !READ && !SEQS) {
+    if (slow) {  // CTA-uniform
+#pragma unroll 1
+        for (int t = 0; t < n; ++t) token(t, std::true_type());
+    } else if constexpr (KIND != MAMBA2 && NC == 4 && DK == 128 && !READ && !SEQS) {
+        // (two tokens per iteration only where the registers allow it without spilling: the
+        // plain update of dk = 128 heads)
 #pragma unroll 2
-        for (int t = 0; t < n; ++t) token(t);
+        for (int t = 0; t < n; ++t) token(t, std::false_type());
     } else {
-        for (int t = 0; t < n; ++t) token(t);
+        for (int t = 0; t < n; ++t) token(t, std::false_type());
     }
 
     // final scale
@@ -261,14 +310,17 @@ update_window_kernel(ST *__restrict__ S, float *__restrict__ P, const float *__r
 
     // shared memory, each array a multiple of 4 floats: dot vectors, update
     // vectors (KDA), values, final scale(s), per-token scalars
+    const int n4 = (n + 3) & ~3;
     float *sk = smem;                                      // [n][DK]
     float *su = sk + (size_t)n * DK;                       // [n][DK] (KDA)
     float *sv = su + (KIND == KDA ? (size_t)n * DK : 0);   // [n][dv]
     float *sg = sv + (size_t)n * dv;                       // [DK]
     float *sut = sg + DK;                                  // [r][DK]: the head's basis rows
     float *ss1 = sut + (size_t)r * DK;                     // [n4]: b_t / g_t (Mamba-2: 1 / g_t)
-    float *ss2 = ss1 + ((n + 3) & ~3);                     // [n4]: b_t
-    float *sq = ss2 + ((n + 3) & ~3);                      // [DK]: the last step's query (when read)
+    float *ss2 = ss1 + n4;                                 // [n4]: b_t
+    float *sa = ss2 + n4;                                  // [n4]: a_t (the plain path)
+    int *sflag = reinterpret_cast<int *>(sa + n4);         // [4]: this head takes the plain path
+    float *sq = sa + n4 + 4;                               // [DK]: the last step's query (when read)
 
     // 1. the state goes in flight first, straight into registers
     float s[NC][EPL];
@@ -292,11 +344,16 @@ update_window_kernel(ST *__restrict__ S, float *__restrict__ P, const float *__r
             }
             const float p0 = warp_prefix_product(a0, lane);
             const float p1 = warp_prefix_product(a1, lane) * __shfl_sync(FULL, p0, 31);
-            if (lane < n) { ss1[lane] = b0 / p0; ss2[lane] = b0; }
-            if (lane + 32 < n) { ss1[lane + 32] = b1 / p1; ss2[lane + 32] = b1; }
+            // every g_t in range: the fold; otherwise the plain recurrence for this head
+            const bool slow = !__all_sync(FULL, (lane >= n || fold_ok(p0)) && (lane + 32 >= n || fold_ok(p1)));
+            if (lane < n) { ss1[lane] = slow ? b0 : b0 / p0; ss2[lane] = b0; sa[lane] = a0; }
+            if (lane + 32 < n) { ss1[lane + 32] = slow ? b1 : b1 / p1; ss2[lane + 32] = b1; sa[lane + 32] = a1; }
             const float g_lo = __shfl_sync(FULL, p0, (n >= 1 && n <= 32) ? n - 1 : 31);
             const float g_hi = __shfl_sync(FULL, p1, n > 32 ? n - 33 : 0);
-            if (lane == 0) sg[0] = n == 0 ? 1.f : (n <= 32 ? g_lo : g_hi);
+            if (lane == 0) {
+                sg[0] = (n == 0 || slow) ? 1.f : (n <= 32 ? g_lo : g_hi);
+                sflag[0] = slow;
+            }
         }
         stage_rows<QT>(kbuf, DK, (size_t)head * W * DK, DK, n, sk, nullptr, tid, nthr);
         __syncthreads();
@@ -307,23 +364,37 @@ update_window_kernel(ST *__restrict__ S, float *__restrict__ P, const float *__r
         stage_rows<float>(abuf, DK, (size_t)head * W * DK, DK, n, su, nullptr, tid, nthr);
         for (int t = tid; t < n; t += nthr) ss2[t] = bbuf[(size_t)head * W + t];
         __syncthreads();
-        // per key channel: g_{t,i} = a_{1,i} ... a_{t,i}; dot vector k g_t (over k),
-        // update vector b k / g_t (over the decay it replaces)
+        // per key channel: g_{t,i} = a_{1,i} ... a_{t,i}, all in range for the fold
+        bool bad = false;
         for (int i = tid; i < DK; i += nthr) {
             float gam = 1.f;
             for (int t = 0; t < n; ++t) {
                 gam *= su[t * DK + i];
-                const float k = sk[t * DK + i];
-                sk[t * DK + i] = k * gam;
-                su[t * DK + i] = ss2[t] * k * (1.f / gam);
+                bad |= !fold_ok(gam);
             }
-            sg[i] = gam;
+        }
+        if (__syncthreads_or(bad)) {  // the plain recurrence: raw keys and decay rows stay as staged
+            for (int i = tid; i < DK; i += nthr) sg[i] = 1.f;
+            if (tid == 0) sflag[0] = 1;
+        } else {
+            // dot vector k g_t (over k), update vector b k / g_t (over the decay it replaces)
+            for (int i = tid; i < DK; i += nthr) {
+                float gam = 1.f;
+                for (int t = 0; t < n; ++t) {
+                    gam *= su[t * DK + i];
+                    const float k = sk[t * DK + i];
+                    sk[t * DK + i] = k * gam;
+                    su[t * DK + i] = ss2[t] * k * (1.f / gam);
+                }
+                sg[i] = gam;
+            }
+            if (tid == 0) sflag[0] = 0;
         }
     }
     __syncthreads();
 
-    apply_store_refresh<KIND, DK, ST, NC, READ, SEQS>(s, sk, su, sv, sg, sut, ss2, sq, S, P, o, head, dv, r, r, n,
-                                          c0, l, lane);
+    apply_store_refresh<KIND, DK, ST, NC, READ, SEQS>(s, sk, su, sv, sg, sut, ss2, sa, sq, S, P, o, head, dv, r, r,
+                                                      n, sflag[0] != 0, c0, l, lane);
 }
 
 // ---------------------------------------------------------------------------
@@ -343,7 +414,7 @@ __host__ __device__ inline int up16(int x) { return (x + 15) & ~15; }
 struct PerLayout {
     int stage_bytes, st, kr, vr, ar, qr;  // inside a stage: state, raw k, raw v, raw decay (KDA), raw query
     int stages;                           // first stage (NS stages follow, stage_bytes apart)
-    int sk, su, sv, sg, sut, ss2, sq, total;
+    int sk, su, sv, sg, sut, ss2, sa, sq, total;
 };
 
 __host__ __device__ inline PerLayout per_layout(int kind, int DK, int dv, int r, int n, int sbytes, int qbytes,
@@ -364,6 +435,7 @@ __host__ __device__ inline PerLayout per_layout(int kind, int DK, int dv, int r,
     L.sg = off; off += up16(DK * 4);
     L.sut = off; off += up16(r * DK * 4);
     L.ss2 = off; off += up16(n * 4);
+    L.sa = off; off += kind == KDA ? 0 : up16(n * 4);
     L.sq = off; off += read ? up16(DK * 4) : 0;
     L.total = off;
     return L;
@@ -406,6 +478,7 @@ update_window_persistent(ST *__restrict__ S, float *__restrict__ P, const float 
     float *sg = reinterpret_cast<float *>(smem + L.sg);
     float *sut = reinterpret_cast<float *>(smem + L.sut);
     float *ss2 = reinterpret_cast<float *>(smem + L.ss2);
+    float *sa = reinterpret_cast<float *>(smem + L.sa);
     float *sq = reinterpret_cast<float *>(smem + L.sq);
     const int state_bytes = dv * DK * (int)sizeof(ST);
     const int kbytes = n * DK * (int)sizeof(QT), vbytes = n * dv * (int)sizeof(QT);
@@ -499,19 +572,23 @@ update_window_persistent(ST *__restrict__ S, float *__restrict__ P, const float 
         }
         const QT *kr = reinterpret_cast<const QT *>(sb + L.kr);
         const QT *vr = reinterpret_cast<const QT *>(sb + L.vr);
+        bool slow = false;  // this head takes the plain recurrence (made CTA-uniform below)
         if (KIND != KDA) {
             // every warp forms g_t = a_1 ... a_t itself (prefix product over lanes t, t + 32)
             const float p0 = warp_prefix_product(a0, lane);
             const float p1 = warp_prefix_product(a1, lane) * __shfl_sync(FULL, p0, 31);
-            const float s_lo = b0 / p0, s_hi = b1 / p1;  // b_t / g_t
+            slow = !__all_sync(FULL, (lane >= n || fold_ok(p0)) && (lane + 32 >= n || fold_ok(p1)));
+            const float s_lo = slow ? b0 : b0 / p0, s_hi = slow ? b1 : b1 / p1;  // b_t / g_t (plain: b_t)
             if (warp == 0) {
                 const float g_lo = __shfl_sync(FULL, p0, (n >= 1 && n <= 32) ? n - 1 : 31);
                 const float g_hi = __shfl_sync(FULL, p1, n > 32 ? n - 33 : 0);
-                if (lane == 0) sg[0] = n == 0 ? 1.f : (n <= 32 ? g_lo : g_hi);
+                if (lane == 0) sg[0] = (n == 0 || slow) ? 1.f : (n <= 32 ? g_lo : g_hi);
                 if (KIND == GDN) {
                     if (lane < n) ss2[lane] = b0;
                     if (lane + 32 < n) ss2[lane + 32] = b1;
                 }
+                if (lane < n) sa[lane] = a0;
+                if (lane + 32 < n) sa[lane + 32] = a1;
             }
             for (int idx = tid * 4; idx < n * DK; idx += nthr * 4) {
                 float f[4];
@@ -540,6 +617,7 @@ update_window_persistent(ST *__restrict__ S, float *__restrict__ P, const float 
                 float gam = 1.f;
                 for (int t = 0; t < n; ++t) {
                     gam *= ar[t * DK + i];
+                    slow |= !fold_ok(gam);
                     const float bt = __shfl_sync(__activemask(), t < 32 ? b0 : b1, t & 31);
                     const float k = ld1(kr + t * DK + i);
                     sk[t * DK + i] = k * gam;
@@ -554,20 +632,30 @@ update_window_persistent(ST *__restrict__ S, float *__restrict__ P, const float 
             }
         }
         if (w + 1 < w_end) load_scalars(w + 1, a0, a1, b0, b1);  // in flight behind this head
-        __syncthreads();  // the stage is consumed; the fp32 staging is ready
-        if (tid == 0 && w + ns < w_end) issue(w + ns, stage);
+        // the fp32 staging is ready; one decision for the CTA
+        slow = __syncthreads_or(slow);
+        if (KIND == KDA && slow) {  // the plain recurrence: raw keys and decay rows, from the still-intact stage
+            const float *ar = reinterpret_cast<const float *>(sb + L.ar);
+            for (int idx = tid; idx < n * DK; idx += nthr) {
+                sk[idx] = ld1(kr + idx);
+                su[idx] = ar[idx];
+            }
+            for (int i = tid; i < DK; i += nthr) sg[i] = 1.f;
+            __syncthreads();
+        }
+        if (tid == 0 && w + ns < w_end) issue(w + ns, stage);  // the stage is consumed
 
         if (!SEQS || head >= 0)  // CTA-uniform
-            apply_store_refresh<KIND, DK, ST, NC, READ, SEQS>(s, sk, su, sv, sg, sut, ss2, sq, S, P, o, head, dv, r,
-                                                        RANKED ? ranked_rows(rank, h, r) : r, n, c0, l,
-                                                        lane);
+            apply_store_refresh<KIND, DK, ST, NC, READ, SEQS>(s, sk, su, sv, sg, sut, ss2, sa, sq, S, P, o, head, dv,
+                                                              r, RANKED ? ranked_rows(rank, h, r) : r, n, slow, c0,
+                                                              l, lane);
     }
 }
 
 static size_t update_smem_bytes(const sketchssm_dims &d, int n) {
     const size_t n4 = (n + 3) & ~3;
     const size_t fl = (size_t)n * d.dk * (d.kind == SKSSM_KDA ? 2 : 1) + (size_t)n * d.dv + d.dk +
-                      (size_t)d.r * d.dk + 2 * n4 + d.dk;
+                      (size_t)d.r * d.dk + 3 * n4 + 4 + d.dk;
     return fl * sizeof(float);
 }
 
@@ -592,12 +680,7 @@ int launch_update_window(const sketchssm_dims &d, void *S, float *P, const float
             if (L.total <= LIMIT) {
                 auto kern = update_window_persistent<KIND, DK, ST, QT, PER_NC, READ, SEQS, RANKED>;
                 const int threads = d.dv * 8 / PER_NC;
-                static bool opted_in = false;
-                if (!opted_in) {
-                    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LIMIT) != cudaSuccess)
-                        return SKSSM_ERR_CUDA;
-                    opted_in = true;
-                }
+                if (allow_max_smem(reinterpret_cast<const void *>(kern)) != SKSSM_OK) return SKSSM_ERR_CUDA;
                 int sms = 0, per_sm = 0;
                 if (sm_count(&sms) != SKSSM_OK ||
                     blocks_per_sm(reinterpret_cast<const void *>(kern), threads, L.total, &per_sm) != SKSSM_OK)
@@ -617,12 +700,7 @@ int launch_update_window(const sketchssm_dims &d, void *S, float *P, const float
             const size_t smem = update_smem_bytes(d, n);
             if (smem > (size_t)LIMIT) return SKSSM_ERR_DIMS;
             auto kern = update_window_kernel<KIND, DK, ST, QT, UPD_NC, READ, SEQS>;
-            static bool opted_in = false;
-            if (!opted_in) {
-                if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LIMIT) != cudaSuccess)
-                    return SKSSM_ERR_CUDA;
-                opted_in = true;
-            }
+            if (allow_max_smem(reinterpret_cast<const void *>(kern)) != SKSSM_OK) return SKSSM_ERR_CUDA;
             kern<<<NH, threads, smem, stream>>>(static_cast<ST *>(S), P, U, static_cast<const QT *>(k),
                                                 static_cast<const QT *>(v), alpha, beta, static_cast<const QT *>(q),
                                                 o, d.B, d.H, d.dv, d.r, n, d.W, seqs, n_seqs);

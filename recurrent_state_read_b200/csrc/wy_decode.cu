@@ -256,13 +256,7 @@ int launch_decode_wy(const sketchssm_dims &d, const float *P, const float *R, co
                     (size_t)WY_WARPS * (j * (SL::KB + SL::VB + SL::AB) + (size_t)d.W * ((d.W + 3) & ~3) * 4);
                 if (smem > 227 * 1024) return SKSSM_ERR_DIMS;
                 auto kern = decode_wy_kernel<KIND, DK, DV, QT>;
-                static bool opted_in = false;
-                if (!opted_in) {
-                    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-                        cudaSuccess)
-                        return SKSSM_ERR_CUDA;
-                    opted_in = true;
-                }
+                if (allow_max_smem(reinterpret_cast<const void *>(kern)) != SKSSM_OK) return SKSSM_ERR_CUDA;
                 kern<<<grid, WY_WARPS * 32, smem, stream>>>(P, R, static_cast<const QT *>(q),
                                                              static_cast<const QT *>(k), static_cast<const QT *>(v),
                                                              alpha, beta, G, o, d.B, d.H, d.r, j, d.W);

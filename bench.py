@@ -556,6 +556,16 @@ def measure_workload(cfg, dev, stream, clocks, barrier, steps, warmup, peak):
     kernels = {"update_window": kernel_entry(bm["update"], t_upd, steps, peak),
                "decode_step": kernel_entry(bm["decode_avg"], t_dec, steps * W, peak),
                "fullread_decode": kernel_entry(bm["fullread"], t_f, steps * W, peak)}
+    if cfg.kind == "gdn" and cfg.W <= 16 and cfg.r <= 16 and cfg.state_dtype == "f32":
+        # the alternative update with the rank-n increment on the tensor cores, same windows
+        St, Pt = S.clone(), P.clone()
+        g_tc = [capture_graph(lambda b=b: rs.sketchssm_update_window_tc(d, St, Pt, U, b.k, b.v, b.alpha, b.beta, W),
+                              stream) for b in bufs]
+        t_tc, _ = timed_windows([g_tc], steps, warmup, stream, clocks, barrier)
+        del g_tc, St, Pt
+        kernels["update_window_tc"] = kernel_entry(bm["update"], t_tc, steps, peak)
+        kernels["update_window_tc"]["note"] = ("sketchssm_update_window_tc: chunked form, rank-n increment on "
+                                               "tcgen05 (not the default path)")
     dominant = "update_window" if t_upd >= t_dec else "decode_step"
     value, value_f = tok_steps / t_s, tok_steps / t_f
     speedup = value / value_f

@@ -135,6 +135,23 @@ int sketchssm_update_window_read(const sketchssm_dims *dims, void *S, float *P, 
                                  int n_tokens, const void *q, float *o, void *stream);
 
 /*
+ * sketchssm_update_window_tc -- sketchssm_update_window for Gated DeltaNet with the
+ * window's tokens applied in chunked (WY) form and the rank-n state increment on the
+ * tensor cores (tcgen05.mma kind::tf32, operands in shared memory, the increment in
+ * tensor memory), the state moved by TMA tiled copies.  Same results as
+ * sketchssm_update_window up to fp32 rounding (W~ is split into two TF32 terms, keys
+ * are exact in TF32).  Applies to SKSSM_GDN with dk = dv = 128, fp32 state, bf16
+ * q/k/v, 1 <= n_tokens <= 16 and r <= 16 (at W <= 16); other sizes return
+ * SKSSM_ERR_DIMS (use sketchssm_update_window).  An alternative implementation of the
+ * same step, not the default: on the Gated DeltaNet workload it measured slower than
+ * sketchssm_update_window.
+ * Arguments and other errors as sketchssm_update_window (n_tokens >= 1).
+ */
+int sketchssm_update_window_tc(const sketchssm_dims *dims, void *S, float *P, const float *U,
+                               const void *k, const void *v, const float *alpha, const float *beta,
+                               int n_tokens, void *stream);
+
+/*
  * sketchssm_decode_step -- one decode step inside a window, reading only the sketch.
  * Defines: SketchSSM abstract (each decode step combines the sketch vectors with
  * query-dependent coefficients instead of reading the full state); digest

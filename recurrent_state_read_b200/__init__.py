@@ -32,6 +32,7 @@ EXPORTS = (
     "sketchssm_version",
     "sketchssm_update_window",
     "sketchssm_update_window_read",
+    "sketchssm_update_window_tc",
     "sketchssm_decode_step",
     "sketchssm_decode_step_seq",
     "sketchssm_update_window_seqs",
@@ -83,6 +84,7 @@ def library() -> ctypes.CDLL:
         lib.sketchssm_version.restype = i
         lib.sketchssm_update_window.argtypes = [D, P, P, P, P, P, P, P, i, P]
         lib.sketchssm_update_window_read.argtypes = [D, P, P, P, P, P, P, P, i, P, P, P]
+        lib.sketchssm_update_window_tc.argtypes = [D, P, P, P, P, P, P, P, i, P]
         lib.sketchssm_decode_step.argtypes = [D, P, P, P, P, P, P, P, i, P, P]
         lib.sketchssm_decode_step_seq.argtypes = [D, P, P, P, P, P, P, P, P, i, P, P]
         lib.sketchssm_update_window_seqs.argtypes = [D, P, P, P, P, P, P, P, i, P, i, P, P, i, P]
@@ -102,7 +104,8 @@ def library() -> ctypes.CDLL:
         lib.sketchssm_selftest_wait_giveup.argtypes = [ctypes.c_uint, P]
         lib.sketchssm_selftest_wait_giveup.restype = i
         lib.sketchssm_device_error_count.restype = i
-        for f in ("sketchssm_update_window", "sketchssm_update_window_read", "sketchssm_decode_step",
+        for f in ("sketchssm_update_window", "sketchssm_update_window_read", "sketchssm_update_window_tc",
+                  "sketchssm_decode_step",
                   "sketchssm_replay_decode_step", "sketchssm_decode_step_seq", "sketchssm_update_window_seqs",
                   "sketchssm_calibrate_basis_ranked", "sketchssm_update_window_ranked",
                   "sketchssm_decode_step_ranked", "sketchssm_decode_step_wy", "sketchssm_fullread_decode",
@@ -170,6 +173,19 @@ def sketchssm_update_window(d: sketchssm_dims, S, P, U, k, v, alpha, beta, n_tok
     _check("sketchssm_update_window",
            library().sketchssm_update_window(ctypes.byref(d), *args, *toks, int(n_tokens),
                                              ctypes.c_void_p(_stream(stream))))
+
+
+def sketchssm_update_window_tc(d: sketchssm_dims, S, P, U, k, v, alpha, beta, n_tokens: int, stream=None):
+    """sketchssm_update_window for Gated DeltaNet with the rank-n state increment on the tensor cores
+    (dk = dv = 128, fp32 state, bf16 q/k/v, 1 <= n_tokens <= 16, r <= 16)."""
+    NH = d.B * d.H
+    args = (_ptr(S, "S", NH * d.dv * d.dk, _dt(d.state_dtype)),
+            None if P is None else _ptr(P, "P", NH * d.dv * d.r, torch.float32),
+            None if U is None else _ptr(U, "U", d.H * d.dk * d.r, torch.float32))
+    toks = _token_ptrs(d, d.W, k, v, alpha, beta)
+    _check("sketchssm_update_window_tc",
+           library().sketchssm_update_window_tc(ctypes.byref(d), *args, *toks, int(n_tokens),
+                                                ctypes.c_void_p(_stream(stream))))
 
 
 def sketchssm_update_window_read(d: sketchssm_dims, S, P, U, k, v, alpha, beta, n_tokens: int, q, o,

@@ -84,6 +84,18 @@ int sketchssm_update_window_read(const sketchssm_dims *d, void *S, float *P, con
                                 (cudaStream_t)stream);
 }
 
+int sketchssm_update_window_tc(const sketchssm_dims *d, void *S, float *P, const float *U, const void *k,
+                               const void *v, const float *alpha, const float *beta, int n_tokens, void *stream) {
+    int rc = check_dims(d);
+    if (rc) return rc;
+    if (!S || (P && !U)) return SKSSM_ERR_NULL;
+    if (n_tokens < 1 || n_tokens > d->W) return SKSSM_ERR_RANGE;
+    if ((rc = check_tokens(d, k, v, alpha, beta))) return rc;
+    if (!aligned(S, 16) || !aligned(P, 16) || !aligned(U, 16)) return SKSSM_ERR_ALIGN;
+    rc = launch_update_window_tc(*d, S, P, P ? U : nullptr, k, v, alpha, beta, n_tokens, (cudaStream_t)stream);
+    return rc == TC_NOT_APPLICABLE ? SKSSM_ERR_DIMS : rc;
+}
+
 int sketchssm_decode_step(const sketchssm_dims *d, const float *P, const float *R, const void *q,
                           const void *k, const void *v, const float *alpha, const float *beta, int j,
                           float *o, void *stream) {

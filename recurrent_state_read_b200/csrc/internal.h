@@ -50,8 +50,14 @@ inline int launch_status() {
 int launch_update_window(const sketchssm_dims &d, void *S, float *P, const float *U, const void *k,
                          const void *v, const float *alpha, const float *beta, int n_tokens, const void *q, float *o,
                          const int *seqs, int n_seqs, int sm_share, const int *rank, cudaStream_t stream);
+// The Gated DeltaNet window update on the tensor cores (update_window_tc.cu) where it applies;
+// TC_NOT_APPLICABLE otherwise (the caller runs the CUDA-core kernel).
+constexpr int TC_NOT_APPLICABLE = 1;
+int launch_update_window_tc(const sketchssm_dims &d, void *S, float *P, const float *U, const void *k,
+                            const void *v, const float *alpha, const float *beta, int n_tokens, cudaStream_t stream);
 // Counts of bounded in-kernel waits that gave up (window update, decode step); reset clears them.
 int update_wait_giveups(bool reset, unsigned *count);
+int update_tc_giveups(bool reset, unsigned *count);
 int decode_wait_giveups(bool reset, unsigned *count);
 
 // Opt a kernel into the largest dynamic shared memory (227 KB) on the current device.  The

@@ -718,6 +718,12 @@ int launch_update_window(const sketchssm_dims &d, void *S, float *P, const float
     });
 }
 
-int update_wait_giveups(bool reset, unsigned *count) { return read_counter(&g_update_wait_giveups, reset, count); }
+int update_wait_giveups(bool reset, unsigned *count) {
+    unsigned tc = 0;
+    if (read_counter(&g_update_wait_giveups, reset, count) != SKSSM_OK || update_tc_giveups(reset, &tc) != SKSSM_OK)
+        return SKSSM_ERR_CUDA;
+    *count += tc;
+    return SKSSM_OK;
+}
 
 }  // namespace skssm

@@ -197,3 +197,31 @@ def test_schedules_edges(case):
     assert max(e_ss, e_sf, e_p) <= s_tol, (e_ss, e_sf, e_p)
     assert max(e_os, e_of) <= o_tol, (e_os, e_of)
     assert rs.sketchssm_device_error_count(1) == 0
+
+
+TC_EDGES = ["reset", "tiny", "beta0", "k0"]
+
+
+@pytest.mark.parametrize("what", TC_EDGES)
+def test_update_window_tc_edges(what):
+    """sketchssm_update_window_tc (Gated DeltaNet, state increment on the tensor cores) on the same
+    edge cases: it multiplies decays and never divides by them, so a zero or vanishing decay needs
+    no special path there; results against the oracle's window update."""
+    import recurrent_state_read_b200 as rs
+
+    cfg, d, S0, U, R, toks = _setup("gdn", what, 128, 128, 8, 16, torch.float32, torch.bfloat16)
+    B, H = d.B, d.H
+    Uh = oracle.per_head(U, H, np.arange(B * H))
+    ft = flat_tokens(toks[0])
+    win = to_window(to_device(toks[0]))
+    rs.sketchssm_device_error_count(1)
+    S = to_gpu_state(S0, B, H)
+    P = torch.full((B, H, 128, 8), float("nan"), device="cuda")
+    rs.sketchssm_update_window_tc(d, S, P, U.transpose(1, 2).contiguous().cuda(), win["k"], win["v"],
+                                  win["alpha"], win["beta"], 16)
+    torch.cuda.synchronize()
+    Sref, Pref = oracle.update_window("gdn", S0, Uh, ft["k"], ft["v"], ft["alpha"], ft["beta"])
+    assert torch.isfinite(S).all() and torch.isfinite(P).all()
+    assert state_err(to_logical(S), Sref) <= STATE_TOL
+    assert state_err(P.reshape(B * H, 128, 8).double().cpu().numpy(), Pref) <= STATE_TOL
+    assert rs.sketchssm_device_error_count(1) == 0

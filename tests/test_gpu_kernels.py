@@ -58,6 +58,7 @@ CASES = [
     ("kda", 128, 128, 8, 16, torch.bfloat16, torch.bfloat16),
     ("gdn", 64, 64, 4, 8, torch.bfloat16, torch.float32),
     ("kda", 128, 128, 128, 64, torch.float32, torch.float32),  # largest layout: one CTA per head
+    ("gdn", 128, 128, 4, 24, torch.float32, torch.float32),    # tensor-core update, fp32 tokens
 ]
 
 
@@ -240,6 +241,38 @@ def test_update_window_many_heads_per_cta(kind):
                                           ft["alpha"][sl], None if ft["beta"] is None else ft["beta"][sl])
         assert state_err(to_logical(S), Sref) <= STATE_TOL, n
         assert state_err(P.reshape(B * H, dv, r).double().cpu().numpy(), Pref) <= STATE_TOL, n
+
+
+TC_PIPE = [(16, 8), (16, 13), (8, 4), (16, 16), (4, 1)]
+
+
+@pytest.mark.parametrize("case", TC_PIPE, ids=[f"W{c[0]}-r{c[1]}" for c in TC_PIPE])
+def test_update_window_tc_pipeline(case):
+    """sketchssm_update_window_tc, the Gated DeltaNet update with the state increment on the tensor
+    cores (dk = dv = 128, fp32 state, bf16 keys), over 2100 heads (B=7, H=300): each persistent CTA
+    runs ~15 heads through its state stages, reusing stages, token buffers and barrier phases,
+    across changes of h; full and partial windows, ranks that need padding.  Every head is checked."""
+    import recurrent_state_read_b200 as rs
+
+    W, r = case
+    cfg, d, S0, U, R, tok = _setup("gdn", 128, 128, r, W, torch.float32, torch.bfloat16, B=7, H=300, seed=11)
+    B, H = d.B, d.H
+    Uh = oracle.per_head(U, H, np.arange(B * H))
+    ft = flat_tokens(tok)
+    dev = to_window(to_device(tok))
+    Ug = U.transpose(1, 2).contiguous().cuda()
+    rs.sketchssm_device_error_count(1)
+    for n in sorted({1, min(7, W), W // 2 + 1, W}):
+        S = to_gpu_state(S0, B, H)
+        P = torch.full((B, H, 128, r), float("nan"), device="cuda")
+        rs.sketchssm_update_window_tc(d, S, P, Ug, dev["k"], dev["v"], dev["alpha"], dev["beta"], n)
+        torch.cuda.synchronize()
+        sl = slice(0, n)
+        Sref, Pref = oracle.update_window("gdn", S0, Uh, ft["k"][sl], ft["v"][sl], ft["alpha"][sl], ft["beta"][sl])
+        es = state_err(to_logical(S), Sref)
+        ep = state_err(P.reshape(B * H, 128, r).double().cpu().numpy(), Pref)
+        assert es <= STATE_TOL and ep <= STATE_TOL, (n, es, ep)
+    assert rs.sketchssm_device_error_count(1) == 0
 
 
 @pytest.mark.parametrize("kind", ["mamba2", "gdn", "kda"])
@@ -439,3 +472,18 @@ def test_bounded_wait_gives_up_and_the_context_survives():
     torch.cuda.synchronize()
     assert torch.isfinite(o).all()
     assert rs.sketchssm_device_error_count(1) == 0
+
+
+def test_update_window_tc_not_applicable():
+    """Sizes outside the tensor-core update's envelope are rejected before any launch."""
+    import recurrent_state_read_b200 as rs
+
+    cfg, d, S0, U, R, tok = _setup("kda", 128, 128, 8, 16, torch.float32, torch.bfloat16)
+    dev = to_window(to_device(tok))
+    S = to_gpu_state(S0, d.B, d.H)
+    P = torch.zeros(d.B, d.H, 128, 8, device="cuda")
+    with pytest.raises(rs.SketchSSMError):
+        rs.sketchssm_update_window_tc(d, S, P, U.transpose(1, 2).contiguous().cuda(), dev["k"], dev["v"],
+                                      dev["alpha"], dev["beta"], 16)
+    torch.cuda.synchronize()
+    assert torch.equal(S, to_gpu_state(S0, d.B, d.H))  # nothing was launched

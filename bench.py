@@ -513,6 +513,36 @@ def approx_error(d, S, P, U, R, buf, tok, dev):
     return float(torch.linalg.vector_norm((out - out_f).double()) / torch.linalg.vector_norm(out_f.double()))
 
 
+def basis_ablation(cfg, d, S, P, U, R, q_cal, bufs, toks, stream, clocks, barrier, steps, warmup, weighted):
+    """The sketch path with the query-PCA basis (sketchssm_calibrate_query_pca: top-r query directions,
+    no state weighting) beside the state-weighted basis: approximation error on the first window and
+    the sketch window's throughput with each.  `weighted` holds the state-weighted basis's figures."""
+    import torch
+
+    import recurrent_state_read_b200 as rs
+
+    dc = dims_of(cfg, B=1)
+    Up, Rp = torch.empty_like(U), torch.empty_like(R)
+    rs.sketchssm_calibrate_query_pca(dc, q_cal, Up, Rp)
+    Sp, Pp = S.clone(), torch.empty_like(P)
+    rs.sketchssm_update_window(d, Sp, Pp, Up, None, None, None, None, 0)
+    approx = approx_error(d, Sp, Pp, Up, Rp, bufs[0], toks[0], S.device)
+    W = cfg.W
+    out = torch.empty(W, cfg.B, cfg.H, cfg.dv, device=S.device)
+    g_dec = [capture_graph(lambda b=b: [rs.sketchssm_decode_step(d, Pp, Rp, b.q[j - 1], b.k, b.v, b.alpha, b.beta,
+                                                                 j, out[j - 1]) for j in range(1, W + 1)], stream)
+             for b in bufs]
+    g_upd = [capture_graph(lambda b=b: rs.sketchssm_update_window(d, Sp, Pp, Up, b.k, b.v, b.alpha, b.beta, W),
+                           stream) for b in bufs]
+    t_s, _ = timed_windows([g_dec, g_upd], steps, warmup, stream, clocks, barrier)
+    del g_dec, g_upd, Sp, Pp
+    return {"rank": cfg.r, "state_weighted": weighted,
+            "query_pca": {"approx_rel_l2_first_window": approx, "value": steps * cfg.B * W / t_s, "unit": UNIT,
+                          "steps": steps},
+            "note": "query PCA: U = R^T = the top-r eigenvectors of the calibration queries' second moment "
+                    "(sketchssm_calibrate_query_pca); same kernels and traffic, only the basis differs"}
+
+
 def measure_workload(cfg, dev, stream, clocks, barrier, steps, warmup, peak):
     """One workload's sketch path (decode steps + window update), full-read path and ReplaySSM-style
     path, each over the same NWIN windows, with per-kernel rooflines, the traffic ratios and the
@@ -527,7 +557,8 @@ def measure_workload(cfg, dev, stream, clocks, barrier, steps, warmup, peak):
     bm = bytes_model(cfg)
     S0 = prefill_state(cfg, dev)
     S_cal = calibration_states(cfg, dev)
-    U, R = calibrate(cfg, S_cal, wl.calibration_queries(cfg, device=dev), dev)
+    q_cal = wl.calibration_queries(cfg, device=dev)
+    U, R = calibrate(cfg, S_cal, q_cal, dev)
     del S_cal
     bufs, toks = decode_windows(cfg, dev)
     W = cfg.W
@@ -569,6 +600,11 @@ def measure_workload(cfg, dev, stream, clocks, barrier, steps, warmup, peak):
     dominant = "update_window" if t_upd >= t_dec else "decode_step"
     value, value_f = tok_steps / t_s, tok_steps / t_f
     speedup = value / value_f
+    ablation = None
+    if cfg.r == 8:
+        ablation = basis_ablation(cfg, d, S, P, U, R, q_cal, bufs, toks, stream, clocks, barrier,
+                                  max(3, steps // 3), warmup,
+                                  {"approx_rel_l2_first_window": approx, "value": value, "unit": UNIT})
     state_ratio = (2 * W * bm["S"]) / (2 * bm["S"] + (W + 1) * bm["P"])
     return {
         "workload": config_json(cfg)["workload"], "value": value, "unit": UNIT, "steps": steps, "warmup": warmup,
@@ -588,6 +624,7 @@ def measure_workload(cfg, dev, stream, clocks, barrier, steps, warmup, peak):
             "gate_on_state_bytes": {"bar": 0.8 * state_ratio, "met": speedup >= 0.8 * state_ratio},
             "gate_on_measured_bytes": measured_gate(cfg, speedup),
             "approx_rel_l2_first_window": approx},
+        **({"basis_ablation": ablation} if ablation else {}),
     }
 
 
@@ -711,7 +748,7 @@ def run_ours(args):
         head_rank = torch.empty(cfg.H, dtype=torch.int32, device=dev)
         lam = torch.empty(cfg.H, cfg.r, dtype=torch.float64, device=dev)
         rs.sketchssm_calibrate_basis_ranked(dc, q_cal, S_cal, args.rank_avg, Uk, Rk, head_rank, lam)
-    del S_cal, P_cal, q_cal
+    del S_cal, P_cal
 
     # NWIN distinct windows of decode tokens
     bufs, toks = [], []
@@ -1052,6 +1089,9 @@ def run_ours(args):
     if world == 1 and not args.no_workloads:
         del g_st
         g_st = None
+        extra["basis_ablation"] = basis_ablation(
+            cfg, d, S, P, U, R, q_cal, bufs, toks, stream, clocks, barrier, max(3, args.workload_steps // 3), 3,
+            {"approx_rel_l2_first_window": approx, "value": value, "unit": UNIT})
         torch.cuda.empty_cache()
         extra["workloads"] = {}
         for name, wcfg in (("gdn", wl.workload(2)), ("kda_r4", wl.workload(3, r=4)), ("kda_r8", wl.workload(3, r=8)),

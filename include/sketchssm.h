@@ -347,6 +347,25 @@ int sketchssm_calibrate_basis(const sketchssm_dims *dims, const float *q_cal, in
                               void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * sketchssm_calibrate_query_pca -- the unweighted basis that the state weighting
+ * is compared against: the top-r principal directions of the calibration
+ * queries, ignoring the states.  SketchSSM abstract: the method's query
+ * approximation is state-weighted; this is that approximation with the state
+ * weight G replaced by the identity, so U = V_r, the eigenvectors of
+ *     C = (1/Nq) sum_n q_n q_n^T
+ * with the r largest eigenvalues, and R = V_r^T (orthogonal projection, R U = I).
+ * Same fp64 kernels as sketchssm_calibrate_basis (Cholesky of I, Jacobi on C).
+ *   q_cal  in  [H][Nq][dk] fp32, Nq >= 1
+ *   U, R   out [H][r][dk] fp32
+ *   workspace: at least sketchssm_calibrate_workspace_bytes(dims, Nq, 1) bytes,
+ *              256-byte aligned, caller-owned.
+ * Offline.  Errors: ERR_NULL, ERR_DIMS, ERR_DTYPE, ERR_RANGE, ERR_ALIGN,
+ * ERR_WORKSPACE, ERR_CUDA.
+ */
+int sketchssm_calibrate_query_pca(const sketchssm_dims *dims, const float *q_cal, int Nq, float *U,
+                                  float *R, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * sketchssm_calibrate_basis_ranked -- the offline calibration with a rank per head
  * under an average-rank budget.  SketchSSM abstract and digest: the traffic
  * reduction is quoted at an average sketch rank of 8, so ranks may differ across

@@ -29,7 +29,7 @@ from typing import Dict, Optional
 import numpy as np
 
 from . import calibration  # noqa: F401
-from .calibration import calibrate, calibrate_heads  # noqa: F401
+from .calibration import calibrate, calibrate_heads, query_pca, query_pca_heads  # noqa: F401
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "sketchssm_oracle.c")

@@ -82,6 +82,29 @@ def calibrate_heads(S_cal: np.ndarray, q_cal: np.ndarray, r: int, ridge: float =
     return np.stack(Us), np.stack(Rs)
 
 
+# ---------------------------------------------------------------------------
+# Query PCA, the unweighted alternative that the state weighting is measured
+# against.  The abstract calls the method's approximation state-weighted; the
+# plain alternative ignores the states and keeps the r principal directions of
+# the calibration queries: U = the eigenvectors of C with the r largest
+# eigenvalues (ties by index), R = U^T, the orthogonal projection onto their span.
+
+
+def query_pca(q_cal: np.ndarray, r: int):
+    """One head: U [dk, r] orthonormal, R = U^T [r, dk]."""
+    lam, V = np.linalg.eigh(gram_queries(q_cal))
+    order = np.argsort(-lam, kind="stable")[:r]
+    U = V[:, order]
+    return U, U.T.copy()
+
+
+def query_pca_heads(q_cal: np.ndarray, r: int):
+    """All heads: q_cal [H, Nq, dk] -> U [H, dk, r], R [H, r, dk]."""
+    q_cal = np.asarray(q_cal, dtype=np.float64)
+    pairs = [query_pca(q_cal[h], r) for h in range(q_cal.shape[0])]
+    return np.stack([u for u, _ in pairs]), np.stack([rr for _, rr in pairs])
+
+
 def objective(G: np.ndarray, C: np.ndarray, U: np.ndarray, R: np.ndarray) -> float:
     """Averaged squared read error tr(C (I - U R)^T G (I - U R)) of a basis/map pair."""
     E = np.eye(G.shape[0]) - U @ R

@@ -42,6 +42,7 @@ EXPORTS = (
     "sketchssm_calibrate_basis",
     "sketchssm_calibrate_basis_noalloc",
     "sketchssm_calibrate_basis_ranked",
+    "sketchssm_calibrate_query_pca",
     "sketchssm_update_window_ranked",
     "sketchssm_decode_step_ranked",
     "sketchssm_decode_step_wy",
@@ -97,6 +98,7 @@ def library() -> ctypes.CDLL:
         lib.sketchssm_calibrate_basis_noalloc.argtypes = [D, P, i, P, i, ctypes.c_double, P, P, P]
         lib.sketchssm_calibrate_basis_ranked.argtypes = [D, P, i, P, i, ctypes.c_double, i, P, P, P, P, P,
                                                          ctypes.c_size_t, P]
+        lib.sketchssm_calibrate_query_pca.argtypes = [D, P, i, P, P, P, ctypes.c_size_t, P]
         lib.sketchssm_update_window_ranked.argtypes = [D, P, P, P, P, P, P, P, P, i, P]
         lib.sketchssm_decode_step_ranked.argtypes = [D, P, P, P, P, P, P, P, P, i, P, P]
         lib.sketchssm_decode_step_wy.argtypes = [D, P, P, P, P, P, P, P, i, P, P, P]
@@ -109,7 +111,8 @@ def library() -> ctypes.CDLL:
                   "sketchssm_replay_decode_step", "sketchssm_decode_step_seq", "sketchssm_update_window_seqs",
                   "sketchssm_calibrate_basis_ranked", "sketchssm_update_window_ranked",
                   "sketchssm_decode_step_ranked", "sketchssm_decode_step_wy", "sketchssm_fullread_decode",
-                  "sketchssm_calibrate_basis", "sketchssm_calibrate_basis_noalloc"):
+                  "sketchssm_calibrate_basis", "sketchssm_calibrate_basis_noalloc",
+                  "sketchssm_calibrate_query_pca"):
             getattr(lib, f).restype = i
         _lib = lib
     return _lib
@@ -292,6 +295,21 @@ def sketchssm_calibrate_basis(d: sketchssm_dims, q_cal, S_cal, U, R, workspace=N
     _check("sketchssm_calibrate_basis", library().sketchssm_calibrate_basis(
         ctypes.byref(d), _ptr(q_cal, "q_cal", d.H * Nq * d.dk, torch.float32), int(Nq),
         _ptr(S_cal, "S_cal", Ns * d.H * d.dv * d.dk, _dt(d.state_dtype)), int(Ns), float(ridge),
+        _ptr(U, "U", d.H * d.dk * d.r, torch.float32), _ptr(R, "R", d.H * d.r * d.dk, torch.float32),
+        _ptr(workspace, "workspace"), ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+        ctypes.c_void_p(_stream(stream))))
+
+
+def sketchssm_calibrate_query_pca(d: sketchssm_dims, q_cal, U, R, workspace=None, stream=None):
+    """Query-PCA basis (no state weighting): q_cal [H,Nq,dk] fp32 -> U, R [H,r,dk] with U = R the
+    top-r principal directions of each head's calibration queries.  Workspace as
+    sketchssm_calibrate_basis with Ns = 1."""
+    Nq = q_cal.shape[1]
+    need = sketchssm_calibrate_workspace_bytes(d, Nq, 1)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q_cal.device)
+    _check("sketchssm_calibrate_query_pca", library().sketchssm_calibrate_query_pca(
+        ctypes.byref(d), _ptr(q_cal, "q_cal", d.H * Nq * d.dk, torch.float32), int(Nq),
         _ptr(U, "U", d.H * d.dk * d.r, torch.float32), _ptr(R, "R", d.H * d.r * d.dk, torch.float32),
         _ptr(workspace, "workspace"), ctypes.c_size_t(workspace.numel() * workspace.element_size()),
         ctypes.c_void_p(_stream(stream))))

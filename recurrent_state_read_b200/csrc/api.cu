@@ -220,6 +220,18 @@ int sketchssm_calibrate_basis(const sketchssm_dims *d, const float *q_cal, int N
     return launch_calibrate(*d, q_cal, Nq, S_cal, Ns, ridge, U, R, workspace, (cudaStream_t)stream);
 }
 
+int sketchssm_calibrate_query_pca(const sketchssm_dims *d, const float *q_cal, int Nq, float *U, float *R,
+                                  void *workspace, size_t workspace_bytes, void *stream) {
+    int rc = check_dims(d);
+    if (rc) return rc;
+    if (!q_cal || !U || !R) return SKSSM_ERR_NULL;
+    if (Nq < 1 || (int64_t)Nq * d->H >= (int64_t)1 << 31) return SKSSM_ERR_RANGE;
+    if (!workspace || workspace_bytes < calibrate_workspace_bytes(*d, Nq, 1)) return SKSSM_ERR_WORKSPACE;
+    if (!aligned(q_cal, 16) || !aligned(U, 16) || !aligned(R, 16) || !aligned(workspace, 256))
+        return SKSSM_ERR_ALIGN;
+    return launch_calibrate(*d, q_cal, Nq, nullptr, 1, 0.0, U, R, workspace, (cudaStream_t)stream);
+}
+
 int sketchssm_calibrate_basis_ranked(const sketchssm_dims *d, const float *q_cal, int Nq, const void *S_cal, int Ns,
                                      double ridge, int r_avg, float *U, float *R, int32_t *rank, double *lam,
                                      void *workspace, size_t workspace_bytes, void *stream) {

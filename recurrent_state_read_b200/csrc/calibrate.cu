@@ -19,6 +19,10 @@
 //                 back substitution for U, and R = V_r^T L^T.
 // U is written as basis rows, U_rows[h][m][i] = U[i][m], like R.
 // Workspace (caller-owned): G/L, C, T/V, each [H][dk][dk] fp64.
+//
+// Query PCA (the unweighted basis the state weighting is measured against): no
+// calibration states, G = I, so L = I, U = V_r holds the top-r eigenvectors of
+// C and R = V_r^T is the orthogonal projection onto their span.
 #include <math.h>
 
 #include "common.cuh"
@@ -306,6 +310,14 @@ int launch_rank_basis(const sketchssm_dims &d, int r_avg, const double *lam, flo
     return launch_status();
 }
 
+// G[h] = I for every head (the query-PCA calibration's state weight).
+__global__ void identity_kernel(double *__restrict__ G, int dk, size_t n) {
+    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x) {
+        const int ij = (int)(e % ((size_t)dk * dk));
+        G[e] = (ij / dk == ij % dk) ? 1.0 : 0.0;
+    }
+}
+
 size_t calibrate_workspace_bytes(const sketchssm_dims &d, int, int) {
     return 3 * (size_t)d.H * d.dk * d.dk * sizeof(double);
 }
@@ -323,6 +335,7 @@ int launch_calibrate(const sketchssm_dims &d, const float *q_cal, int Nq, const 
 
 // Heads [h0, h0 + hc) only, with a workspace sized for hc heads: G and C (fp64 Gram
 // kernels), then the per-head basis, with every head-indexed pointer offset to h0.
+// S_cal == nullptr selects G = I (query PCA; ridge is then irrelevant).
 int launch_calibrate_heads(const sketchssm_dims &d, const float *q_cal, int Nq, const void *S_cal,
                            int Ns, double ridge, float *U, float *R, void *workspace, int h0, int hc,
                            cudaStream_t stream, double *lam) {
@@ -334,7 +347,10 @@ int launch_calibrate_heads(const sketchssm_dims &d, const float *q_cal, int Nq, 
         const dim3 ggrid((DK / 32) * (DK / 32), hc);
         const size_t sh = (size_t)d.dv * DK, sb = (size_t)d.H * d.dv * DK;
         const size_t s_off = (size_t)h0 * d.dv * DK;
-        if (d.state_dtype == SKSSM_F32)
+        if (!S_cal) {
+            const size_t n = (size_t)hc * DK * DK;
+            identity_kernel<<<(int)((n + 255) / 256 < 2048 ? (n + 255) / 256 : 2048), 256, 0, stream>>>(G, DK, n);
+        } else if (d.state_dtype == SKSSM_F32)
             gram_kernel<float, DK><<<ggrid, 256, 0, stream>>>(static_cast<const float *>(S_cal) + s_off, sh,
                                                               sb, d.dv, Ns * d.dv, 1.0 / Ns, G);
         else

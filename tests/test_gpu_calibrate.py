@@ -60,6 +60,28 @@ def test_calibrate_matches_oracle(cid, n_seq, n_tokens, n_q, r):
         assert j_gpu <= j_ref * (1 + 1e-4) + 1e-12 * np.trace(G @ C), (h, j_gpu, j_ref)
 
 
+@pytest.mark.parametrize("cid,r", [(1, 8), (2, 8), (3, 16), (0, 4)])
+def test_query_pca_matches_oracle(cid, r):
+    """sketchssm_calibrate_query_pca: the projector U R onto the top-r query directions, R U = I
+    and R = U^T, against the oracle's eigh-based query PCA on the same queries."""
+    import recurrent_state_read_b200 as rs
+
+    cfg = wl.workload(cid, H=min(wl.CONFIGS[cid].H, 5), r=r)
+    q_cal = wl.calibration_queries(cfg, n=1024)
+    U_ref, R_ref = oracle.query_pca_heads(q_cal.double().numpy(), r)
+    d = rs.dims(cfg.kind, 1, cfg.H, cfg.dk, cfg.dv, r, cfg.W, torch.float32, cfg.torch_qkv_dtype)
+    U = torch.full((cfg.H, r, cfg.dk), float("nan"), device="cuda")
+    R = torch.full((cfg.H, r, cfg.dk), float("nan"), device="cuda")
+    rs.sketchssm_calibrate_query_pca(d, q_cal.cuda().contiguous(), U, R)
+    torch.cuda.synchronize()
+    U, R = U.transpose(1, 2).double().cpu().numpy(), R.double().cpu().numpy()
+    for h in range(cfg.H):
+        Pi, Pi_ref = U[h] @ R[h], U_ref[h] @ R_ref[h]
+        assert np.abs(Pi - Pi_ref).max() <= 1e-5, (h, np.abs(Pi - Pi_ref).max())
+        np.testing.assert_allclose(R[h] @ U[h], np.eye(r), atol=1e-5)
+        np.testing.assert_allclose(R[h], U[h].T, atol=1e-6)
+
+
 def test_calibrate_bf16_states():
     import recurrent_state_read_b200 as rs
 

@@ -182,13 +182,10 @@ def test_config3_kda(r):
     _sampled(wl.workload(3, r=r))
 
 
-SWEEP = [
-    dict(B=64, r=4, W=4, state_dtype="f32"),
-    dict(B=1024, r=32, W=32, state_dtype="f32"),
-    dict(B=256, r=16, W=8, state_dtype="bf16"),
-    dict(B=1024, r=8, W=16, state_dtype="bf16"),
-    dict(B=64, r=32, W=32, state_dtype="bf16"),
-]
+# every (r, W) of the GDN sweep at B = 64 in both state dtypes, the B = 1024 corners, and one B = 256 point
+SWEEP = ([dict(B=64, r=r, W=W, state_dtype=dt) for dt in ("f32", "bf16") for r in (4, 8, 16, 32) for W in (4, 8, 16, 32)]
+         + [dict(B=1024, r=r, W=W, state_dtype=dt) for dt in ("f32", "bf16") for r in (4, 32) for W in (4, 32)]
+         + [dict(B=256, r=16, W=8, state_dtype="bf16")])
 
 
 @pytest.mark.parametrize("pt", SWEEP, ids=[f"B{p['B']}-r{p['r']}-W{p['W']}-{p['state_dtype']}" for p in SWEEP])

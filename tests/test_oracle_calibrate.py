@@ -204,3 +204,52 @@ def test_ranked_basis_is_the_truncated_full_basis():
         if rh:  # the same projector as a rank-r_h calibration of that head alone
             Ur, Rr = cal.calibrate(S[:, h], q[h], int(rh))
             np.testing.assert_allclose(U[h] @ R[h], Ur @ Rr, atol=1e-9)
+
+
+# ---- query PCA (the unweighted basis the state weighting is compared with) ----
+
+def test_query_pca_axis_aligned_closed_form():
+    """Queries +-s_i e_i give C = diag(s_i^2) / dk exactly: the basis is the r axes with the
+    largest s_i, in descending order, and R = U^T."""
+    dk, r = 9, 4
+    s = np.array([0.5, 3.0, 1.0, 7.0, 0.1, 2.0, 5.0, 0.7, 4.0])
+    q = np.concatenate([np.diag(s), -np.diag(s)])
+    U, R = cal.query_pca(q, r)
+    top = [3, 6, 8, 1]  # s = 7, 5, 4, 3
+    np.testing.assert_allclose(np.abs(U), np.eye(dk)[:, top], atol=1e-12)
+    np.testing.assert_array_equal(R, U.T)
+
+
+def test_query_pca_is_the_svd_projection():
+    """Eckart-Young: the unweighted residual mean ||q - U R q||^2 of the PCA basis is the sum of
+    the trailing squared singular values of the query matrix / Nq, and the projector is the
+    span of the top right singular vectors (numpy's SVD, a different routine from eigh)."""
+    rng = np.random.default_rng(31)
+    dk, r, Nq = 14, 5, 300
+    q = rng.standard_normal((Nq, dk)) * np.linspace(2.5, 0.3, dk)[None, :] @ np.linalg.qr(
+        rng.standard_normal((dk, dk)))[0]
+    U, R = cal.query_pca(q, r)
+    np.testing.assert_allclose(R @ U, np.eye(r), atol=1e-12)
+    sv, Vt = np.linalg.svd(q, full_matrices=False)[1:]
+    np.testing.assert_allclose(U @ R, Vt[:r].T @ Vt[:r], atol=1e-10)
+    resid = np.mean(np.sum((q - q @ (U @ R).T) ** 2, axis=1))
+    np.testing.assert_allclose(resid, np.sum(sv[r:] ** 2) / Nq, rtol=1e-10)
+
+
+def test_query_pca_equals_weighted_basis_under_isotropic_states():
+    """The state-weighted calibration with S S^T the same multiple of I for every state has the
+    same projector as the query-PCA basis."""
+    rng = np.random.default_rng(32)
+    dk, r = 10, 3
+    O = np.linalg.qr(rng.standard_normal((dk, dk)))[0]
+    S = np.stack([O * 0.8, O[:, ::-1] * 0.8])
+    q = rng.standard_normal((400, dk)) * np.linspace(2.0, 0.5, dk)[None, :]
+    Uw, Rw = cal.calibrate(S, q, r, ridge=0.0)
+    Up, Rp = cal.query_pca_heads(q[None], r)
+    np.testing.assert_allclose(Uw @ Rw, Up[0] @ Rp[0], atol=1e-9)
+    # and the state weighting wins on a non-isotropic state population
+    S2, q2 = _data(rng, 40, 300, dk, 6, rank=6, noise=0.3)
+    U2, R2 = cal.calibrate(S2, q2, r, ridge=0.0)
+    Up2, Rp2 = cal.query_pca(q2, r)
+    G, C = cal.gram_states(S2), cal.gram_queries(q2)
+    assert cal.objective(G, C, U2, R2) < cal.objective(G, C, Up2, Rp2)

@@ -162,3 +162,32 @@ def test_bf16_state_rounds_once_per_window(orc):
     Sx, _ = orc.update_window("gdn", S0, U, K, V, A, Bt)
     np.testing.assert_array_equal(S, orc.round_bf16(Sx))
     np.testing.assert_allclose(P, np.einsum("nic,nim->ncm", S, U), rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("kind", KINDS)
+def test_bf16_state_rounds_after_every_step(orc, kind):
+    """The full-read path with a bf16 state stores the state after every token: the
+    token's read sees the fp64 update of the stored (rounded) state, and the stored
+    state is that update rounded to bf16.  Restated with dense transition matrices
+    stepped in fp64 and torch's bf16 conversion after each step."""
+    import torch
+
+    def bf16(x):
+        return torch.from_numpy(np.ascontiguousarray(x)).float().to(torch.bfloat16).double().numpy()
+
+    rng = np.random.default_rng(11)
+    N, dk, dv, T = 2, 6, 5, 9
+    S0 = bf16(rng.standard_normal((N, dk, dv)))
+    K, V, A, Bt, Q = _tokens(rng, kind, T, N, dk, dv)
+    S, O = orc.exact_steps(kind, S0, K, V, A, Bt, Q, bf16_state=True)
+    for n in range(N):
+        Sd = S0[n].copy()
+        for t in range(T):
+            b = 1.0 if kind == "mamba2" else Bt[t, n]
+            Sd = _dense_M(kind, K[t, n], A[t, n], b) @ Sd + b * np.outer(K[t, n], V[t, n])
+            np.testing.assert_allclose(O[t, n], Sd.T @ Q[t, n], rtol=1e-12, atol=1e-12)
+            Sd = bf16(Sd)
+        np.testing.assert_array_equal(S[n], Sd)
+    # the rounding is not the identity on these values: an unrounded run differs
+    Sx, Ox = orc.exact_steps(kind, S0, K, V, A, Bt, Q)
+    assert np.abs(Sx - S).max() > 1e-4 and np.abs(Ox - O).max() > 1e-4

@@ -130,6 +130,9 @@ def hbm_peak():
 KERNEL_SOURCES = {
     "decode_step": ("decode_step.cu", "decode_common.cuh", "common.cuh", "state_tile.cuh", "internal.h"),
     "update_window": ("update_window.cu", "common.cuh", "state_tile.cuh", "internal.h"),
+    # every kernel of a sketch window and of a full-read window
+    "window": ("decode_step.cu", "decode_common.cuh", "update_window.cu", "fullread.cu", "common.cuh",
+               "state_tile.cuh", "internal.h"),
 }
 
 
@@ -484,7 +487,7 @@ def measured_gate(cfg, speedup):
             if ":" in line and not line.startswith(" "):
                 k, v = line.split(":", 1)
                 kv[k.strip()] = v.strip()
-    if (kv.get("csrc_sha256") or "").split()[:1] != [csrc_hash()] or kv.get("workload_key") != workload_key(cfg):
+    if (kv.get("csrc_sha256") or "").split()[:1] != [csrc_hash("window")] or kv.get("workload_key") != workload_key(cfg):
         return None
     try:
         full = float(kv["fullread_dram_bytes_per_token_step"])
@@ -1091,7 +1094,8 @@ def run_ours(args):
         g_st = None
         extra["basis_ablation"] = basis_ablation(
             cfg, d, S, P, U, R, q_cal, bufs, toks, stream, clocks, barrier, max(3, args.workload_steps // 3), 3,
-            {"approx_rel_l2_first_window": approx, "value": value, "unit": UNIT})
+            {"approx_rel_l2_first_window": approx,
+             "value": whole_job_rate(args.steps * cfg.B * cfg.W, world, t_sketch), "unit": UNIT})
         torch.cuda.empty_cache()
         extra["workloads"] = {}
         for name, wcfg in (("gdn", wl.workload(2)), ("kda_r4", wl.workload(3, r=4)), ("kda_r8", wl.workload(3, r=8)),

@@ -130,9 +130,12 @@ def hbm_peak():
 KERNEL_SOURCES = {
     "decode_step": ("decode_step.cu", "decode_common.cuh", "common.cuh", "state_tile.cuh", "internal.h"),
     "update_window": ("update_window.cu", "common.cuh", "state_tile.cuh", "internal.h"),
-    # every kernel of a sketch window and of a full-read window
+    "update_window_tc": ("update_window_tc.cu", "common.cuh", "internal.h"),
+    # every kernel of a sketch window and of a full-read window (with the tensor-core update: window_tc)
     "window": ("decode_step.cu", "decode_common.cuh", "update_window.cu", "fullread.cu", "common.cuh",
                "state_tile.cuh", "internal.h"),
+    "window_tc": ("decode_step.cu", "decode_common.cuh", "update_window_tc.cu", "fullread.cu", "common.cuh",
+                  "state_tile.cuh", "internal.h"),
 }
 
 
@@ -158,7 +161,8 @@ def profiled_traffic(kernel_tag, cfg):
             if ":" in line and not line.startswith(" "):
                 k, v = line.split(":", 1)
                 kv[k.strip()] = v.strip()
-    kernel = "decode_step" if kernel_tag.startswith("decode_step") else "update_window"
+    kernel = ("decode_step" if kernel_tag.startswith("decode_step")
+              else "update_window_tc" if tc_update(cfg) else "update_window")
     if (kv.get("csrc_sha256") or "").split()[:1] != [csrc_hash(kernel)] or kv.get("workload_key") != workload_key(cfg):
         return None
     try:
@@ -487,7 +491,8 @@ def measured_gate(cfg, speedup):
             if ":" in line and not line.startswith(" "):
                 k, v = line.split(":", 1)
                 kv[k.strip()] = v.strip()
-    if (kv.get("csrc_sha256") or "").split()[:1] != [csrc_hash("window")] or kv.get("workload_key") != workload_key(cfg):
+    srcs = "window_tc" if tc_update(cfg) else "window"
+    if (kv.get("csrc_sha256") or "").split()[:1] != [csrc_hash(srcs)] or kv.get("workload_key") != workload_key(cfg):
         return None
     try:
         full = float(kv["fullread_dram_bytes_per_token_step"])
@@ -546,6 +551,13 @@ def basis_ablation(cfg, d, S, P, U, R, q_cal, bufs, toks, stream, clocks, barrie
                     "(sketchssm_calibrate_query_pca); same kernels and traffic, only the basis differs"}
 
 
+def tc_update(cfg):
+    """Whether sketchssm_update_window runs this workload's windows on the tensor cores (Gated DeltaNet,
+    dk = dv = 128, fp32 state, bf16 q/k/v, r <= 16, 12 <= W <= 16 tokens per window)."""
+    return (cfg.kind == "gdn" and cfg.dk == 128 and cfg.dv == 128 and cfg.state_dtype == "f32"
+            and cfg.qkv_dtype == "bf16" and cfg.r <= 16 and 12 <= cfg.W <= 16)
+
+
 def measure_workload(cfg, dev, stream, clocks, barrier, steps, warmup, peak):
     """One workload's sketch path (decode steps + window update), full-read path and ReplaySSM-style
     path, each over the same NWIN windows, with per-kernel rooflines, the traffic ratios and the
@@ -590,16 +602,9 @@ def measure_workload(cfg, dev, stream, clocks, barrier, steps, warmup, peak):
     kernels = {"update_window": kernel_entry(bm["update"], t_upd, steps, peak),
                "decode_step": kernel_entry(bm["decode_avg"], t_dec, steps * W, peak),
                "fullread_decode": kernel_entry(bm["fullread"], t_f, steps * W, peak)}
-    if cfg.kind == "gdn" and cfg.W <= 16 and cfg.r <= 16 and cfg.state_dtype == "f32":
-        # the alternative update with the rank-n increment on the tensor cores, same windows
-        St, Pt = S.clone(), P.clone()
-        g_tc = [capture_graph(lambda b=b: rs.sketchssm_update_window_tc(d, St, Pt, U, b.k, b.v, b.alpha, b.beta, W),
-                              stream) for b in bufs]
-        t_tc, _ = timed_windows([g_tc], steps, warmup, stream, clocks, barrier)
-        del g_tc, St, Pt
-        kernels["update_window_tc"] = kernel_entry(bm["update"], t_tc, steps, peak)
-        kernels["update_window_tc"]["note"] = ("sketchssm_update_window_tc: chunked form, rank-n increment on "
-                                               "tcgen05 (not the default path)")
+    if tc_update(cfg):
+        kernels["update_window"]["path"] = ("tensor cores: chunked form, S_0^T [K; U] and the rank-n increment "
+                                            "on tcgen05 (kind::tf32, split operands)")
     dominant = "update_window" if t_upd >= t_dec else "decode_step"
     value, value_f = tok_steps / t_s, tok_steps / t_f
     speedup = value / value_f
@@ -684,7 +689,8 @@ def run_sweep(dev, stream, clocks, barrier, steps, warmup, peak):
                         "bytes_per_token_step": bm["sketch_step"] / (B * W),
                         "window_GBps": win_gbps, "window_frac": win_gbps / peak,
                         "update_us": upd["us_per_launch"], "update_GBps": upd["GBps"], "update_frac": upd["frac_of_peak"],
-                        "decode_us": dec["us_per_launch"], "decode_GBps": dec["GBps"], "decode_frac": dec["frac_of_peak"]})
+                        "decode_us": dec["us_per_launch"], "decode_GBps": dec["GBps"], "decode_frac": dec["frac_of_peak"],
+                        "update_path": "tensor cores" if tc_update(cfg) else "cuda cores"})
                 if W == 16:  # the full-read path does not depend on W or r
                     d = dims_of(cfgB)
                     bm = bytes_model(cfgB)

@@ -103,6 +103,10 @@ int sketchssm_version(void);
  * decay product underflows or exceeds the fp32 range: such a head is updated
  * token by token instead of through the running decay scale.
  * n_tokens = 0 is a sketch refresh only (S is read, not written).
+ * Implementation: SKSSM_GDN with dk = dv = 128, fp32 state, bf16 q/k/v, r <= 16
+ * and 12 <= n_tokens <= 16 runs the chunked form on the tensor cores (as
+ * sketchssm_update_window_tc, below); every other case runs the token-by-token
+ * kernel on the CUDA cores.  Both give the recurrence's result to fp32 rounding.
  *   S        in/out [B][H][dv][dk] state_dtype
  *   P        out    [B][H][dv][r] fp32; NULL: no sketch refresh (a plain buffered
  *            state update, the window-end write of the ReplaySSM-style path)
@@ -136,15 +140,15 @@ int sketchssm_update_window_read(const sketchssm_dims *dims, void *S, float *P, 
 
 /*
  * sketchssm_update_window_tc -- sketchssm_update_window for Gated DeltaNet with the
- * window's tokens applied in chunked (WY) form and the rank-n state increment on the
- * tensor cores (tcgen05.mma kind::tf32, operands in shared memory, the increment in
- * tensor memory), the state moved by TMA tiled copies.  Same results as
- * sketchssm_update_window up to fp32 rounding (W~ is split into two TF32 terms, keys
- * are exact in TF32).  Applies to SKSSM_GDN with dk = dv = 128, fp32 state, bf16
- * q/k/v, 1 <= n_tokens <= 16 and r <= 16 (at W <= 16); other sizes return
- * SKSSM_ERR_DIMS (use sketchssm_update_window).  An alternative implementation of the
- * same step, not the default: on the Gated DeltaNet workload it measured slower than
- * sketchssm_update_window.
+ * window's tokens applied in chunked (WY) form, both products on the tensor cores
+ * (tcgen05.mma kind::tf32): [X | S_0^T U] = S_0^T [K; U] with the state split into
+ * its TF32 part and remainder, and the rank-n state increment W~^T K with W~ split
+ * the same way, so the result matches the recurrence to fp32 rounding (keys are
+ * exact in TF32).  The state moves by TMA tiled copies.  Applies to SKSSM_GDN with
+ * dk = dv = 128, fp32 state, bf16 q/k/v, 1 <= n_tokens <= 16 and r <= 16; other
+ * sizes return SKSSM_ERR_DIMS.  sketchssm_update_window takes this path by itself
+ * for 12 <= n_tokens <= 16; this entry forces it for any n_tokens >= 1 (below 12
+ * tokens the CUDA-core kernel is faster).
  * Arguments and other errors as sketchssm_update_window (n_tokens >= 1).
  */
 int sketchssm_update_window_tc(const sketchssm_dims *dims, void *S, float *P, const float *U,

@@ -14,35 +14,40 @@
 //     w_t = b_t v_t - b_t g_t x_t - sum_{s<t} b_t gamma_{t,s} (k_t . k_s) w_s,
 //     x_t = S_0^T k_t.
 // Per head (dk = dv = 128, S stored transposed, row c = column c of S):
-//   1. X = S_0^T K^T and S_0^T U^T  fp32 dot products on the CUDA cores (a value
-//                                   channel's row against every key and basis row)
-//   2. the key Gram K K^T and K U^T, fp32, CUDA cores
-//   3. the triangular solve         CUDA cores, one value channel per thread
+//   1. [X | S_0^T U^T] = S_0^T [K; U]   tcgen05.mma kind::tf32, M = 128 (c), N = 16 + 2 RP,
+//                                      K = 128 (i): one pass with the state as it
+//                                      arrived, one with its TF32 remainder
+//   2. the key Gram K K^T and K U^T    fp32 on the CUDA cores, under step 1
+//   3. the triangular solve            CUDA cores, one value channel per thread
 //   4. D^T = W~^T K, W~_s = gamma_{n-1,s} w_s
-//                                   tcgen05.mma kind::tf32, M = 128, N = 128, K = n,
-//                                   both operands in shared memory
-//   5. S_n^T = g_{n-1} S_0^T + D^T, and the sketch without a pass over S_n:
+//                                      tcgen05.mma, M = 128, N = 128, K = n, W~ in
+//                                      tensor memory (A), the keys MN-major (B)
+//   5. S_n^T = g_{n-1} S_0^T + D^T, and the sketch
 //          P = S_n^T U = g_{n-1} S_0^T U + sum_t W~_t (K U^T)_t
-// The tensor cores take the rank-n update (half of the arithmetic); the dot
-// products stay on the CUDA cores because their N (the n tokens) is too narrow:
-// a tcgen05.mma costs ~56 cycles to issue whatever N <= 128 (measured), so the
-// 32 instructions X would need cost more than the dots themselves.
-// fp32 accuracy from the TF32 tensor cores: a TF32 operand keeps the top 11
-// significant bits of an fp32 value, so W~ is split as W~ = hi + lo with hi = W~
-// with its low 13 mantissa bits cleared (exactly TF32) and lo = W~ - hi (exact
-// in fp32; the tensor core keeps its top 11 bits); the keys are bf16, exact in
-// TF32, so D = hi^T K + lo^T K in two passes, off by less than 2^-21 of W~.
+// fp32 accuracy from the TF32 tensor cores.  A TF32 operand keeps the top 11
+// significant bits of an fp32 value: the tensor core drops the 13 low mantissa
+// bits (measured: 1 + 0.75 ulp of TF32 enters as 1).  The state goes in as it
+// arrived (the tensor core takes its TF32 part t(S_0)) and as its remainder
+// S_0 - t(S_0), exact in fp32, of which the tensor core keeps the top 11 bits; the keys are bf16, exact
+// in TF32; the basis rows go in split as U = hi + lo with hi exactly TF32.  So
+// every product of step 1 is off by less than 2^-21 of its terms.  W~ is split
+// the same way for step 4.
 //
-// Data movement: a persistent CTA (one per SM: the shared memory below takes
-// most of the SM) walks a contiguous run of heads in (h, b) order.  Each head's
-// state arrives by four TMA tiled copies (cp.async.bulk.tensor, 128 rows x 32
-// fp32 each, 128-byte swizzle) into one of NS shared-memory stages, one head or
-// more ahead; the tokens arrive by 1-D bulk copies one head ahead.  Each thread
-// keeps its 64 values of S_0 in registers from step 1 to step 5, which writes
-// S_n back into the stage, from where it leaves by TMA tiled stores.  Roles:
-// warp 0 issues the MMAs, warp 1 the copies (and polls their barriers), warp 4
-// (lane t = token t) does the per-token scalars; the other warps sleep in CTA
-// barriers rather than poll.  Tensor memory: D, 128 columns.
+// Data movement: a persistent CTA (one per SM) walks a contiguous run of heads in
+// (h, b) order.  Each head's state arrives by four TMA tiled copies
+// (cp.async.bulk.tensor, 128 rows x 32 fp32 each, 128-byte swizzle) into one of
+// two shared-memory stages, which is the A operand of step 1's first pass, one
+// head ahead.  Each thread keeps its 64 values of S_0 in registers from the split
+// (step 1) to step 5 and writes the remainder into tensor memory, from where the
+// second pass reads it (A operand in tensor memory).  Step 5 writes S_n back
+// into the stage, from where it leaves by TMA tiled stores (a thread per row
+// storing to global memory directly costs one transaction per row per store).
+// The keys and values arrive by 1-D bulk copies one head ahead.  Roles: warp 0
+// issues the MMAs, warp 1 the copies; warps 2, 3, 6 and 7 compute the key Gram,
+// K U^T and the system matrix A[t][s] = b_t gamma_{t,s} (k_t . k_s) under step 1
+// (off the issuers' sub-partitions); warps 0-3 (one value channel per thread)
+// solve, while warp 4 builds the next head's decay products.  Tensor memory (512
+// columns): the remainder (128), [X | S_0^T U] (<= 128), D (128), W~ hi | lo (32).
 // Every wait is bounded; a wait that gives up is counted
 // (sketchssm_device_error_count), the CTA drains what it has in flight (bounded),
 // frees its tensor memory and returns.
@@ -59,45 +64,46 @@ __device__ unsigned g_update_tc_giveups;
 namespace {
 
 constexpr int TC_THREADS = 256;  // 8 warps; warps w and w + 4 share tensor-memory lanes 32 (w % 4) ..
+constexpr int TC_NS = 2;         // state stages
+constexpr int TC_NPAD = 16;      // token rows of the operands (tokens n .. 15 are zero)
 constexpr int TC_PANEL = 128 * 128;    // bytes of one 32-column panel of a head's state (128 rows x 128 B)
 constexpr int TC_STATE = 4 * TC_PANEL;
-constexpr uint32_t TM_COLS = 128;
-constexpr uint32_t TM_D = 0;  // tensor-memory columns of the state increment D
+constexpr uint32_t TM_COLS = 512;
+constexpr uint32_t TM_LO = 0;    // the state's TF32 remainder, 128 columns (A of step 1's second pass)
+constexpr uint32_t TM_D1 = 128;  // [X | S_0^T U hi-part | S_0^T U lo-part], N1 <= 48 columns
+constexpr uint32_t TM_D2 = 256;  // the state increment D^T, 128 columns
+constexpr uint32_t TM_W = 384;   // W~^T hi (16 columns) then lo (16): A of step 4
 constexpr int TC_SMEM_LIMIT = 227 * 1024;
 
 __host__ __device__ inline int round_up(int x, int a) { return (x + a - 1) / a * a; }
+__host__ __device__ constexpr int tc_n1(int rp) { return (TC_NPAD + 2 * rp + 15) / 16 * 16; }
 
 // Shared-memory layout: byte offsets from the 1024-aligned base.
 struct TcLayout {
-    int stages;     // NS x 64 KB: state stages (TMA destination and source), 1024-aligned
-    int wh, wl;     // W~^T hi and lo: 128 rows x 128 B, K-major, 128-byte swizzle (A of step 4)
-    int kbm;        // the keys, MN-major TF32 layout: 4 panels x npad rows x 128 B (B of step 4)
-    int kf;         // the keys, fp32 rows [npad][128] (step 1, 2)
-    int uf;         // the basis rows, fp32 [rp][128] (rows r .. rp-1 zero)
-    int tok;        // two token buffers: k rows then v rows of one head, bf16
+    int stages;     // TC_NS x 64 KB: state stages (TMA destination; A of step 1's first pass)
+    int b1;         // B of step 1: N1 rows [keys (16) | U hi (RP) | U lo (RP) | 0] x 128 fp32, K-major,
+                    // 128-byte swizzle, 4 panels of N1 rows x 128 B
+    int kbm;        // the keys, MN-major TF32 layout: 4 panels x 16 rows x 128 B (B of step 4)
+    int tok;        // two token buffers: 16 key rows then 16 value rows, bf16
     int tok_bytes;  // bytes of one token buffer
-    int xex;        // partial dot products of the second column half: [128][npad + rp]
-    int am;         // A [npad][npad + 1], G [npad][npad + 1], K U^T [npad][rp], b_t g_t, gamma_{n-1,t},
-                    // b_t [npad] each, g
-    int bars;       // mbarriers: NS stages, 2 token buffers, D, drain
+    int am;         // by head parity: A, decay table [2][16][20] each, K U^T [2][16][RP], b_t g_t,
+                    // gamma_{n-1,t}, b_t [2][16] each, g [2]
+    int bars;       // mbarriers: 2 stages, 2 token buffers, step 1, step 4, drain
     int slot;       // tensor-memory base address written by tcgen05.alloc
     int total;      // bytes to request (with slack for aligning the base)
 };
 
-__host__ __device__ inline TcLayout tc_layout(int ns, int npad, int rp, int W) {
+__host__ __device__ inline TcLayout tc_layout(int rp) {
     TcLayout L;
+    const int n1 = tc_n1(rp);
     int o = 0;
-    L.stages = o; o += ns * TC_STATE;
-    L.wh = o; o += 128 * 128;
-    L.wl = o; o += 128 * 128;
-    L.kbm = o; o += npad * 512;
-    L.kf = o; o += npad * 512;
-    L.uf = o; o += rp * 512;
-    L.tok_bytes = round_up(2 * W * 128 * 2, 128);
+    L.stages = o; o += TC_NS * TC_STATE;
+    L.b1 = o; o += round_up(n1 * 512, 1024);
+    L.kbm = o; o += TC_NPAD * 512;
+    L.tok_bytes = 2 * TC_NPAD * 128 * 2;
     L.tok = o; o += 2 * L.tok_bytes;
-    L.xex = o; o += 128 * (npad + rp) * 4;
-    L.am = o; o += round_up((2 * npad * (npad + 1) + npad * rp + 3 * npad + 4) * 4, 16);
-    L.bars = o; o += 8 * (ns + 4);
+    L.am = o; o += round_up((4 * TC_NPAD * (TC_NPAD + 4) + 2 * TC_NPAD * rp + 6 * TC_NPAD + 4) * 4, 16);
+    L.bars = o; o += 8 * (TC_NS + 5);
     L.slot = o; o += 16;
     L.total = o + 1024;
     return L;
@@ -184,8 +190,11 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// fp32 value with the 13 low mantissa bits cleared: what a TF32 operand keeps of it
+// fp32 value with the 13 low mantissa bits cleared: exactly a TF32 value
 __device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float(__float_as_uint(x) & 0xffffe000u); }
+// The TF32 value the tensor core takes of an fp32 operand that is not already TF32 (the state
+// stage): its 13 low mantissa bits dropped.
+__device__ __forceinline__ float tc_tf32(float x) { return tf32_hi(x); }
 
 // Shared-memory matrix descriptors.  K-major, 128-byte swizzle: atoms of 8 rows x 128 B, 1024 B
 // apart (the leading offset is unused); a K step of 8 TF32 values advances the start by 32 B inside
@@ -249,17 +258,38 @@ __device__ __forceinline__ bool elect_one() {
     return pred != 0;
 }
 
-template <int NPAD, int RP>
+// Recursive-halving reduce-scatter of 32 per-lane partials: on return lane l holds in v[0] the sum
+// over the warp of every lane's v[l] (31 shuffles).
+__device__ __forceinline__ void warp_reduce_scatter32(float (&v)[32], int lane) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < o; ++i) {
+            const float send = up ? v[i] : v[i + o];
+            const float keep = up ? v[i + o] : v[i];
+            v[i] = keep + __shfl_xor_sync(FULL, send, o);
+        }
+    }
+}
+
+// 4-wide fp32 dot product
+__device__ __forceinline__ float dot4(float4 a, float4 b) {
+    return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, a.w * b.w)));
+}
+
+template <int RP>
 __global__ void __launch_bounds__(TC_THREADS, 1)
-update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict__ P, const float *__restrict__ U,
-                     const __nv_bfloat16 *__restrict__ kbuf, const __nv_bfloat16 *__restrict__ vbuf,
-                     const float *__restrict__ abuf, const float *__restrict__ bbuf, int B, int H, int r, int n, int W,
-                     int ns) {
+update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict__ P,
+                     const float *__restrict__ U, const __nv_bfloat16 *__restrict__ kbuf,
+                     const __nv_bfloat16 *__restrict__ vbuf, const float *__restrict__ abuf,
+                     const float *__restrict__ bbuf, int B, int H, int r, int n, int W) {
     using QT = __nv_bfloat16;
-    constexpr int npad = NPAD, NX = NPAD + RP, as = NPAD + 1;
+    constexpr int NPAD = TC_NPAD, N1 = tc_n1(RP), as = NPAD + 4;  // rows of A and G: 16-byte aligned
+    constexpr int B1P = N1 * 128;  // bytes of one 32-column panel of B1
     extern __shared__ __align__(1024) unsigned char tc_raw[];
     unsigned char *sm = tc_raw + ((1024 - (smem_u32(tc_raw) & 1023)) & 1023);
-    const TcLayout L = tc_layout(ns, npad, RP, W);
+    const TcLayout L = tc_layout(RP);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int quad = warp & 3, half = warp >> 2;
     const int row = 32 * quad + lane;  // this thread's state row (value channel) and tensor-memory lane
@@ -268,24 +298,22 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
     const int w_begin = blockIdx.x * per, w_end = min(NH, w_begin + per);
     if (w_begin >= w_end) return;  // the whole CTA, before anything is allocated
 
-    uint64_t *bar_s = reinterpret_cast<uint64_t *>(sm + L.bars);  // [ns] state stages
-    uint64_t *bar_t = bar_s + ns;                                 // [2] token buffers
-    uint64_t *bar_c = bar_t + 2;                                  // the state increment D
-    uint64_t *bar_d = bar_c + 1;                                  // the drain after a give-up
+    uint64_t *bar_s = reinterpret_cast<uint64_t *>(sm + L.bars);  // [2] state stages
+    uint64_t *bar_t = bar_s + TC_NS;                              // [2] key buffers
+    uint64_t *bar_1 = bar_t + 2;                                  // step 1 complete
+    uint64_t *bar_4 = bar_1 + 1;                                  // step 4 complete
+    uint64_t *bar_d = bar_4 + 1;                                  // the drain after a give-up
     uint32_t *slot = reinterpret_cast<uint32_t *>(sm + L.slot);
-    float *Am = reinterpret_cast<float *>(sm + L.am);  // [npad][as]: A[t][s] = b_t gamma_{t,s} G[t][s], s < t
-    float *Gm = Am + npad * as;                         // [npad][as]: G[t][s] = k_t . k_s, s < t
-    float *kus = Gm + npad * as;                        // [npad][RP]: (K U^T)[t][m]
-    float *ev = kus + npad * RP;                        // [npad]: b_t g_t
-    float *cv = ev + npad;                              // [npad]: gamma_{n-1,s}
-    float *bv = cv + npad;                              // [npad]: b_t
-    float *gn = bv + npad;                              // [1]:  g_{n-1}
-    float *kf = reinterpret_cast<float *>(sm + L.kf);   // [npad][128]
-    float *uf = reinterpret_cast<float *>(sm + L.uf);   // [RP][128]
-    float *xex = reinterpret_cast<float *>(sm + L.xex);  // [128][NX]
-    unsigned char *kbm = sm + L.kbm;
-    unsigned char *wh = sm + L.wh, *wl = sm + L.wl;
-    const uint32_t kbm_a = smem_u32(kbm), wh_a = smem_u32(wh), wl_a = smem_u32(wl);
+    // per head parity:
+    float *Am = reinterpret_cast<float *>(sm + L.am);  // [2][16][as]: A[t][s] = b_t gamma_{t,s} G[t][s] (s < t, else 0)
+    float *Gam = Am + 2 * NPAD * as;                    // [2][16][as]: b_t gamma_{t,s} (s < t, else 0)
+    float *kus = Gam + 2 * NPAD * as;                   // [2][16][RP]: (K U^T)[t][m]
+    float *ev = kus + 2 * NPAD * RP;                    // [2][16]: b_t g_t
+    float *cv = ev + 2 * NPAD;                          // [2][16]: gamma_{n-1,s}
+    float *bv = cv + 2 * NPAD;                          // [2][16]: b_t
+    float *gn = bv + 2 * NPAD;                          // [2]:  g_{n-1}
+    unsigned char *b1 = sm + L.b1, *kbm = sm + L.kbm;
+    const uint32_t b1_a = smem_u32(b1), kbm_a = smem_u32(kbm);
     const int kbytes = n * 128 * (int)sizeof(QT);
 
     auto head_of = [&](int w) { return (w % B) * H + w / B; };
@@ -302,12 +330,91 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
         const size_t off = (size_t)head_of(w) * W * 128;
         mbar_expect_tx(bar, 2 * kbytes);
         bulk_g2s(tok_of(i), kbuf + off, kbytes, bar);
-        bulk_g2s(tok_of(i) + W * 128 * sizeof(QT), vbuf + off, kbytes, bar);
+        bulk_g2s(tok_of(i) + NPAD * 128 * sizeof(QT), vbuf + off, kbytes, bar);
+    };
+
+    float a_nx = 1.f, b_nx = 0.f;  // warp 4, lane t: a_t and b_t of the next head to build a system for
+    // warp 4: a head's decay table from its token scalars (lane t holds a_t, b_t; lanes >= n: a = 1, b = 0)
+    auto decay_table = [&](float a_l, float b_l, int buf) {
+        const float at = lane < n ? a_l : 1.f, bt = lane < n ? b_l : 0.f;
+        float g = at;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_up_sync(FULL, g, o);
+            if (lane >= o) g *= y;
+        }
+        float sp = at;  // suffix products: sp_s = a_s ... a_31
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_down_sync(FULL, sp, o);
+            if (lane + o < 32) sp *= y;
+        }
+        const float c = __shfl_down_sync(FULL, sp, 1);
+        if (lane < NPAD) {
+            ev[buf * NPAD + lane] = bt * g;
+            bv[buf * NPAD + lane] = bt;
+            cv[buf * NPAD + lane] = c;  // gamma_{n-1,s} = a_{s+1} ... a_{n-1} (a = 1 past n)
+        }
+        const float gl = __shfl_sync(FULL, g, n - 1);
+        if (lane == 0) gn[buf] = gl;
+        float *gm = Gam + buf * NPAD * as;
+        float gam = 1.f;  // gamma_{t,s} for t = lane, s descending
+#pragma unroll
+        for (int s = NPAD - 1; s >= 0; --s) {
+            const float a1 = __shfl_sync(FULL, at, s + 1);
+            if (lane > s) gam *= a1;
+            if (lane < NPAD) gm[lane * as + s] = lane > s && lane < n ? bt * gam : 0.f;
+        }
+    };
+
+    // warps 2, 3, 6, 7 (not the sub-partitions of the MMA and copy issuers): this head's key Gram and
+    // K U^T from the fp32 rows of B1 (keys, U hi and lo), and A = (b_t gamma_{t,s}) o G into buffer buf
+    auto gram_system = [&](int buf) {
+        const int t0 = 4 * ((warp & 1) + (warp >> 1 & 2));  // rows t0 .. t0 + 3
+        // lane l: key channels 4l .. 4l+3 (panel l / 8, chunk l % 8 of its 128-byte rows)
+        const unsigned char *pn = b1 + (lane >> 3) * B1P;
+        auto rowv = [&](int rr) {
+            return *reinterpret_cast<const float4 *>(pn + rr * 128 + ((((lane & 7) ^ rr) & 7) << 4));
+        };
+        float4 ks[NPAD];  // every key row once (rows n .. 15 are zero)
+#pragma unroll
+        for (int j = 0; j < NPAD; ++j) ks[j] = rowv(j);
+        float4 kt[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) kt[j] = rowv(t0 + j);
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {  // rows t0 + 2g, t0 + 2g + 1 against every key row
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = dot4(kt[2 * g + (i >> 4)], ks[i & 15]);
+            warp_reduce_scatter32(v, lane);
+            const int tt = t0 + 2 * g + (lane >> 4), ss = lane & 15;
+            Am[(buf * NPAD + tt) * as + ss] = Gam[(buf * NPAD + tt) * as + ss] * v[0];
+        }
+#pragma unroll
+        for (int m0 = 0; m0 < RP; m0 += 8) {  // K U^T with U = hi + lo, eight basis rows at a time
+            float4 uu[8];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                if (m0 + m < RP) {
+                    const float4 uh = rowv(NPAD + m0 + m), ul = rowv(NPAD + RP + m0 + m);
+                    uu[m] = make_float4(uh.x + ul.x, uh.y + ul.y, uh.z + ul.z, uh.w + ul.w);
+                } else {
+                    uu[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+            float v[32];  // index i = 8 (row) + m
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = dot4(kt[i >> 3], uu[i & 7]);
+            warp_reduce_scatter32(v, lane);
+            const int m = m0 + (lane & 7);
+            if (m < RP) kus[(buf * NPAD + t0 + (lane >> 3)) * RP + m] = v[0];
+        }
     };
 
     if (warp == 0) {
         if (elect_one()) {
-            for (int i = 0; i < ns + 4; ++i) mbar_init(bar_s + i, 1);
+            for (int i = 0; i < TC_NS + 5; ++i) mbar_init(bar_s + i, 1);
             asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         }
         __syncwarp();
@@ -316,6 +423,11 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
+    // the key rows n .. 15 of B1 and of the MN-major keys stay zero for the whole run
+    for (int i = tid; i < (4 * B1P + NPAD * 512) / 16; i += TC_THREADS) {
+        unsigned char *dst = i < 4 * B1P / 16 ? b1 + 16 * i : kbm + 16 * (i - 4 * B1P / 16);
+        *reinterpret_cast<float4 *>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -323,18 +435,18 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
     const uint32_t tlane = tbase + ((uint32_t)(32 * quad) << 16);  // this warp's lanes
 
     // loads issued and not yet waited on, tracked by warp 1 for a drain after a give-up (bit st:
-    // stage st, bit i: token buffer i), with the parity their completion will have
+    // stage st, bit i: key buffer i), with the parity their completion will have
     unsigned pend_s = 0, pend_t = 0, par_s = 0, par_t = 0;
     auto note_state = [&](int w, int st) {
         pend_s |= 1u << st;
-        par_s = (par_s & ~(1u << st)) | ((unsigned)(((w - w_begin) / ns) & 1) << st);
+        par_s = (par_s & ~(1u << st)) | ((unsigned)(((w - w_begin) / TC_NS) & 1) << st);
     };
     auto note_tok = [&](int w, int i) {
         pend_t |= 1u << i;
         par_t = (par_t & ~(1u << i)) | ((unsigned)(((w - w_begin) >> 1) & 1) << i);
     };
     if (warp == 1) {
-        for (int st = 0; st < ns && w_begin + st < w_end; ++st) {
+        for (int st = 0; st < TC_NS && w_begin + st < w_end; ++st) {
             if (elect_one()) issue_state(w_begin + st, st);
             note_state(w_begin + st, st);
         }
@@ -343,255 +455,196 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
         __syncwarp();
     }
     // per-token scalars, prefetched one head ahead by warp 4 (lane t holds token t)
-    float a_nx = 1.f, b_nx = 0.f;
-    if (warp == 4 && lane < n) {
-        a_nx = abuf[(size_t)head_of(w_begin) * W + lane];
-        b_nx = bbuf[(size_t)head_of(w_begin) * W + lane];
+    if (warp == 4) {
+        if (lane < n) {
+            a_nx = abuf[(size_t)head_of(w_begin) * W + lane];
+            b_nx = bbuf[(size_t)head_of(w_begin) * W + lane];
+        }
+        decay_table(a_nx, b_nx, 0);  // the first head's
     }
-    int h_prev = -1;
     bool failed = false;
-    constexpr uint32_t idx_c = idesc_tf32(128, 128, 1);
-    const int kc = (n + 7) >> 3;  // K steps of the state increment
+    int h_prev = -1;
+    constexpr uint32_t idx_1 = idesc_tf32(128, N1, 0);
+    constexpr uint32_t idx_4 = idesc_tf32(128, 128, 1);
+    const int kc = (n + 7) >> 3;  // K steps of step 4
 
     for (int w = w_begin, it = 0; w < w_end; ++w, ++it) {
-        const int st = it % ns, tb = it & 1, ph = it & 1;
+        const int st = it % TC_NS, tb = it & 1, ph = it & 1;
         const int head = head_of(w), h = w / B;
         unsigned char *stage = stage_of(st);
         const unsigned char *tk = tok_of(tb);
-        // the next head's tokens into the other buffer (its last reader, the previous head, is done)
+        // the next head's keys into the other buffer (its last reader, the previous head, is done)
         if (warp == 1 && w + 1 < w_end) {
             fence_proxy_async();
             if (elect_one()) issue_tok(w + 1, tb ^ 1);
             note_tok(w + 1, tb ^ 1);
             __syncwarp();
         }
-        const float a_t = a_nx, b_t = b_nx;
-        if (warp == 4 && w + 1 < w_end && lane < n) {
+        const int db = it & 1;  // this head's decay table
+        if (warp == 4 && w + 1 < w_end && lane < n) {  // the next head's scalars, for its table
             a_nx = abuf[(size_t)head_of(w + 1) * W + lane];
             b_nx = bbuf[(size_t)head_of(w + 1) * W + lane];
         }
-        if (h != h_prev) {  // basis rows of head index h (rows r .. RP-1 zero)
+        if (h != h_prev) {  // basis rows of head index h into B1 rows 16 .. (hi, then lo; rows past r zero)
             for (int i = tid; i < RP * 32; i += TC_THREADS) {
-                const int m = i >> 5;
-                reinterpret_cast<float4 *>(uf)[i] =
-                    (P != nullptr && m < r) ? reinterpret_cast<const float4 *>(U + (size_t)h * r * 128)[i]
-                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+                const int m = i >> 5, c4 = (i & 31) * 4;
+                float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (P != nullptr && m < r) u = reinterpret_cast<const float4 *>(U + ((size_t)h * r + m) * 128)[i & 31];
+                const float4 uh = make_float4(tf32_hi(u.x), tf32_hi(u.y), tf32_hi(u.z), tf32_hi(u.w));
+                const float4 ul = make_float4(u.x - uh.x, u.y - uh.y, u.z - uh.z, u.w - uh.w);
+                unsigned char *pn = b1 + (c4 >> 5) * B1P;
+                *reinterpret_cast<float4 *>(pn + sw128(NPAD + m, c4 & 31)) = uh;
+                *reinterpret_cast<float4 *>(pn + sw128(NPAD + RP + m, c4 & 31)) = ul;
             }
             h_prev = h;
         }
-        // ---- tokens landed: the keys as fp32 rows, and MN-major for step 4 (rows n .. npad-1 zero)
+        // ---- keys and state landed
         bool ok = true;
         if (warp == 1) {
             ok = mbar_wait(bar_t + tb, (it >> 1) & 1);
             pend_t &= ~(1u << tb);
+            if (ok) {
+                ok = mbar_wait(bar_s + st, (it / TC_NS) & 1);
+                pend_s &= ~(1u << st);
+            }
         }
         if (__syncthreads_or(!ok)) { failed = true; break; }
-        for (int i = tid; i < npad * 16; i += TC_THREADS) {
+        // ---- the keys as fp32 rows of B1 (K-major) and of the MN-major operand of step 4
+        for (int i = tid; i < n * 16; i += TC_THREADS) {
             const int t = i >> 4, c8 = (i & 15) * 8;
-            float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            if (t < n) {
-                load4(reinterpret_cast<const QT *>(tk) + t * 128 + c8, x);
-                load4(reinterpret_cast<const QT *>(tk) + t * 128 + c8 + 4, x + 4);
-            }
+            float x[8];
+            load4(reinterpret_cast<const QT *>(tk) + t * 128 + c8, x);
+            load4(reinterpret_cast<const QT *>(tk) + t * 128 + c8 + 4, x + 4);
             const float4 lo4 = make_float4(x[0], x[1], x[2], x[3]), hi4 = make_float4(x[4], x[5], x[6], x[7]);
-            *reinterpret_cast<float4 *>(kf + t * 128 + c8) = lo4;
-            *reinterpret_cast<float4 *>(kf + t * 128 + c8 + 4) = hi4;
-            unsigned char *dst = kbm + (c8 >> 5) * (npad * 128) + sw128_32b(t, c8 & 31);
+            unsigned char *pn = b1 + (c8 >> 5) * B1P;
+            *reinterpret_cast<float4 *>(pn + sw128(t, c8 & 31)) = lo4;
+            *reinterpret_cast<float4 *>(pn + sw128(t, (c8 & 31) + 4)) = hi4;
+            unsigned char *dst = kbm + (c8 >> 5) * (NPAD * 128) + sw128_32b(t, c8 & 31);
             *reinterpret_cast<float4 *>(dst) = lo4;
             *reinterpret_cast<float4 *>(dst + 16) = hi4;
         }
-        fence_proxy_async();  // the MN-major keys are read by the tensor core
+        // ---- the split: this thread's 64 state values into registers, their TF32 remainder into
+        // tensor memory (lane = row, column = key channel)
+        float s0[64];
+#pragma unroll
+        for (int j2 = 0; j2 < 2; ++j2) {
+            const int pnl = 2 * half + j2;
+            uint32_t lo[32];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 f = *reinterpret_cast<const float4 *>(stage + pnl * TC_PANEL + sw128(row, 4 * q));
+                s0[32 * j2 + 4 * q] = f.x; s0[32 * j2 + 4 * q + 1] = f.y;
+                s0[32 * j2 + 4 * q + 2] = f.z; s0[32 * j2 + 4 * q + 3] = f.w;
+                lo[4 * q] = __float_as_uint(f.x - tc_tf32(f.x));
+                lo[4 * q + 1] = __float_as_uint(f.y - tc_tf32(f.y));
+                lo[4 * q + 2] = __float_as_uint(f.z - tc_tf32(f.z));
+                lo[4 * q + 3] = __float_as_uint(f.w - tc_tf32(f.w));
+            }
+            tmem_st32(tlane + TM_LO + 32 * pnl, lo);
+        }
+        tmem_wait_st();
+        fence_proxy_async();  // B1 and the MN-major keys, written here, are read by the tensor core
+        tc_fence_before();
         __syncthreads();
-        // ---- the key Gram (t > s) and K U^T: one dot of two 128-vectors per task, the rows read from a
-        // per-thread starting chunk so that the threads of a warp fall on distinct banks
-        {
-            const int ng = n * (n - 1) / 2;
-            const int rot = tid & 31;
-            for (int task = tid; task < ng + n * RP; task += TC_THREADS) {
-                const float *x, *y;
-                int t, s2;
-                if (task < ng) {
-                    t = 1;
-                    int rem = task;
-                    while (rem >= t) { rem -= t; ++t; }
-                    s2 = rem;
-                    x = kf + t * 128;
-                    y = kf + s2 * 128;
-                } else {
-                    t = (task - ng) / RP;
-                    s2 = (task - ng) % RP;
-                    x = kf + t * 128;
-                    y = uf + s2 * 128;
-                }
-                float2 acc2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                                  make_float2(0.f, 0.f)};
-#pragma unroll 4
-                for (int q = 0; q < 32; ++q) {
-                    const int c = ((q + rot) & 31) * 4;
-                    const float4 a4 = *reinterpret_cast<const float4 *>(x + c);
-                    const float4 b4 = *reinterpret_cast<const float4 *>(y + c);
-                    acc2[q & 3] = fma2(make_float2(a4.x, a4.y), make_float2(b4.x, b4.y), acc2[q & 3]);
-                    acc2[q & 3] = fma2(make_float2(a4.z, a4.w), make_float2(b4.z, b4.w), acc2[q & 3]);
-                }
-                const float dsum = (acc2[0].x + acc2[0].y) + (acc2[1].x + acc2[1].y) + (acc2[2].x + acc2[2].y) +
-                                   (acc2[3].x + acc2[3].y);
-                if (task < ng) Gm[t * as + s2] = dsum;
-                else kus[t * RP + s2] = dsum;
-            }
-        }
-        float at = 1.f, bt = 0.f;  // warp 4: this lane's token scalars (lanes >= n: a = 1, b = 0)
-        if (warp == 4) {  // decay products
-            at = lane < n ? a_t : 1.f;
-            bt = lane < n ? b_t : 0.f;
-            float g = at;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float y = __shfl_up_sync(FULL, g, o);
-                if (lane >= o) g *= y;
-            }
-            float sp = at;  // suffix products: sp_s = a_s ... a_31
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float y = __shfl_down_sync(FULL, sp, o);
-                if (lane + o < 32) sp *= y;
-            }
-            const float c = __shfl_down_sync(FULL, sp, 1);
-            if (lane < npad) {
-                ev[lane] = bt * g;
-                bv[lane] = bt;
-                cv[lane] = lane == 31 ? 1.f : c;  // gamma_{n-1,s} = a_{s+1} ... a_{n-1}
-            }
-            const float gl = __shfl_sync(FULL, g, n - 1);
-            if (lane == 0) *gn = gl;
-        }
-        // ---- state landed
-        if (warp == 1) {
-            ok = mbar_wait(bar_s + st, (it / ns) & 1);
-            pend_s &= ~(1u << st);
-        }
-        if (__syncthreads_or(!ok)) { failed = true; break; }  // (also: the Gram and the scalars are ready)
-        if (warp == 4) {
-            // the system (I + A) w = y, A[t][s] = b_t gamma_{t,s} (k_t . k_s) for s < t (lane t = row t),
-            // then T~ = diag(gamma_{n-1,.}) (I + A)^-1 (lane s = column s), so that W~ = T~ y
-            float gam = 1.f;  // gamma_{t,s} for t = lane, s descending
-#pragma unroll
-            for (int s = NPAD - 2; s >= 0; --s) {
-                const float a1 = __shfl_sync(FULL, at, s + 1);
-                if (lane > s) {
-                    gam *= a1;
-                    if (lane < n) Am[lane * as + s] = bt * gam * Gm[lane * as + s];
-                }
-            }
-            __syncwarp();
-            // column `lane` of (I + A)^-1 by forward substitution; its entries above the diagonal are
-            // zero, so every row sums over all u < t without a test (two partial sums)
-            float tc[NPAD];
-#pragma unroll
-            for (int t = 0; t < NPAD; ++t) {
-                float x0 = t == lane ? 1.f : 0.f, x1 = 0.f;
-                if (t < n) {
-#pragma unroll
-                    for (int u = 0; u < t; u += 2) {
-                        x0 = fmaf(-Am[t * as + u], tc[u], x0);
-                        if (u + 1 < t) x1 = fmaf(-Am[t * as + u + 1], tc[u + 1], x1);
-                    }
-                }
-                tc[t] = t < n ? x0 + x1 : 0.f;
-            }
-            if (lane < NPAD)
-#pragma unroll
-                for (int t = 0; t < NPAD; ++t) Gm[t * as + lane] = t < n ? cv[t] * tc[t] : 0.f;  // T~ over the Gram
-        } else if (warp == 1) {  // the stage of the previous head is refilled once its store has read it
-            if (ns > 1 && it >= 1 && w - 1 + ns < w_end) {
+        if (warp == 1) {  // the previous head's stage, once its store has read it, for the head two ahead
+            if (it >= 1 && w - 1 + TC_NS < w_end) {
                 if (elect_one()) {
                     bulk_wait_read_all();
                     fence_proxy_async();
-                    issue_state(w - 1 + ns, (it - 1) % ns);
+                    issue_state(w - 1 + TC_NS, (it - 1) % TC_NS);
                 }
-                note_state(w - 1 + ns, (it - 1) % ns);
+                note_state(w - 1 + TC_NS, (it - 1) % TC_NS);
                 __syncwarp();
             }
         }
-        // ---- step 1: this thread's 64 state values, dotted with every key and basis row
-        float s0[64];
+        if (warp == 0) {  // ---- step 1: [X | S_0^T U] = S_0^T [K; U], the stage pass and the remainder pass
+            tc_fence_after();
+            // a descriptor's address field is the byte address / 16 (shared addresses < 256 KB: no carry),
+            // so the K steps are offsets added to one base descriptor
+            const uint64_t ad0 = smem_desc_kmajor_sw128(smem_u32(stage)), bd0 = smem_desc_kmajor_sw128(b1_a);
+            if (elect_one()) {
 #pragma unroll
-        for (int j2 = 0; j2 < 2; ++j2)
+                for (int kk = 0; kk < 16; ++kk)  // the stage as it arrived (the tensor core takes its TF32 part)
+                    mma_ss(tbase + TM_D1, ad0 + (((kk >> 2) * TC_PANEL + (kk & 3) * 32) >> 4),
+                           bd0 + (((kk >> 2) * B1P + (kk & 3) * 32) >> 4), idx_1, kk);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const float4 f =
-                    *reinterpret_cast<const float4 *>(stage + (2 * half + j2) * TC_PANEL + sw128(row, 4 * q));
-                s0[32 * j2 + 4 * q] = f.x; s0[32 * j2 + 4 * q + 1] = f.y;
-                s0[32 * j2 + 4 * q + 2] = f.z; s0[32 * j2 + 4 * q + 3] = f.w;
+                for (int kk = 0; kk < 16; ++kk)  // the remainder, from tensor memory
+                    mma_ts(tbase + TM_D1, tbase + TM_LO + 8 * kk, bd0 + (((kk >> 2) * B1P + (kk & 3) * 32) >> 4),
+                           idx_1, 1);
+                mma_commit(bar_1);
             }
-        float xp[NX];
-        {
-            // all NX dot products at once, four channels at a time: every accumulator is independent
-            // (rows past n and basis rows past r are zero in shared memory)
-            float2 a2[NX];
-#pragma unroll
-            for (int j = 0; j < NX; ++j) a2[j] = make_float2(0.f, 0.f);
-            const float *kfh = kf + 64 * half, *ufh = uf + 64 * half;
-#pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                const float2 sa = make_float2(s0[4 * q], s0[4 * q + 1]), sb = make_float2(s0[4 * q + 2], s0[4 * q + 3]);
-#pragma unroll
-                for (int j = 0; j < NX; ++j) {
-                    const float4 v4 = *reinterpret_cast<const float4 *>(
-                        (j < NPAD ? kfh + j * 128 : ufh + (j - NPAD) * 128) + 4 * q);
-                    a2[j] = fma2(sa, make_float2(v4.x, v4.y), a2[j]);
-                    a2[j] = fma2(sb, make_float2(v4.z, v4.w), a2[j]);
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < NX; ++j) xp[j] = a2[j].x + a2[j].y;
+            __syncwarp();
+        } else if ((warp & 2) != 0) {  // ---- step 2 under step 1
+            gram_system(db);
         }
-        if (half == 1)
-#pragma unroll
-            for (int j = 0; j < NX; j += 4)
-                *reinterpret_cast<float4 *>(xex + row * NX + j) = make_float4(xp[j], xp[j + 1], xp[j + 2], xp[j + 3]);
-        __syncthreads();
-        const float g = *gn;
-        // ---- steps 3 and 5 (the sketch): the triangular solve, one value channel per thread (warps 0-3)
+        // ---- step 1 complete
+        if (warp == 0) ok = mbar_wait(bar_1, ph);
+        if (__syncthreads_or(!ok)) { failed = true; break; }
+        const float g = gn[db];
+        // ---- step 3: the triangular solve, one value channel per thread (warps 0-3), and the sketch
         if (half == 0) {
+            tc_fence_after();
+            float xd[N1];
+            {
+                uint32_t d[32];
+                tmem_ld32(tlane + TM_D1, d);
+                tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < NX; j += 4) {
-                const float4 o4 = *reinterpret_cast<const float4 *>(xex + row * NX + j);
-                xp[j] += o4.x; xp[j + 1] += o4.y; xp[j + 2] += o4.z; xp[j + 3] += o4.w;
-            }
-            const QT *vt = reinterpret_cast<const QT *>(tk + W * 128 * sizeof(QT));
-            float y[NPAD], acc[NPAD];
+                for (int j = 0; j < 32; ++j) xd[j] = __uint_as_float(d[j]);
+                if constexpr (N1 > 32) {
 #pragma unroll
-            for (int t = 0; t < NPAD; ++t) y[t] = t < n ? bv[t] * ld1(vt + t * 128 + row) - ev[t] * xp[t] : 0.f;
-            // W~ = T~ y (T~ lower triangular, zero past n)
+                    for (int c0 = 32; c0 < N1; c0 += 16) {
+                        uint32_t e[16];
+                        tmem_ld16(tlane + TM_D1 + c0, e);
+                        tmem_wait_ld();
 #pragma unroll
-            for (int t = 0; t < NPAD; ++t) {
-                float x = 0.f;
-#pragma unroll
-                for (int s = 0; s <= t; ++s) x = fmaf(Gm[t * as + s], y[s], x);
-                acc[t] = x;
-            }
-            // W~ split hi | lo, as row `row` of the A operands of step 4
-#pragma unroll
-            for (int q = 0; q < NPAD / 4; ++q) {
-                float hv[4], lv[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    hv[e] = tf32_hi(acc[4 * q + e]);
-                    lv[e] = acc[4 * q + e] - hv[e];
+                        for (int j = 0; j < 16; ++j) xd[c0 + j] = __uint_as_float(e[j]);
+                    }
                 }
-                *reinterpret_cast<float4 *>(wh + sw128(row, 4 * q)) = make_float4(hv[0], hv[1], hv[2], hv[3]);
-                *reinterpret_cast<float4 *>(wl + sw128(row, 4 * q)) = make_float4(lv[0], lv[1], lv[2], lv[3]);
             }
-            // P = S_n^T U = g S_0^T U + sum_t w~_t (K U^T)_t
+            const QT *vt = reinterpret_cast<const QT *>(tk + NPAD * 128 * sizeof(QT));
+            float wv[NPAD];
+            const float *A = Am + db * NPAD * as;
+#pragma unroll
+            for (int t = 0; t < NPAD; ++t) {  // (I + A) w = y, forward (A[t][s] = 0 for s >= t)
+                // (value rows past n are not copied: their shared memory is not read)
+                float y0 = t < n ? bv[db * NPAD + t] * ld1(vt + t * 128 + row) - ev[db * NPAD + t] * xd[t] : 0.f,
+                      y1 = 0.f;
+#pragma unroll
+                for (int s4 = 0; s4 < t; s4 += 4) {
+                    const float4 a4 = *reinterpret_cast<const float4 *>(A + t * as + s4);
+                    y0 = fmaf(-a4.x, wv[s4], y0);
+                    if (s4 + 1 < t) y1 = fmaf(-a4.y, wv[s4 + 1], y1);
+                    if (s4 + 2 < t) y0 = fmaf(-a4.z, wv[s4 + 2], y0);
+                    if (s4 + 3 < t) y1 = fmaf(-a4.w, wv[s4 + 3], y1);
+                }
+                wv[t] = y0 + y1;
+            }
+#pragma unroll
+            for (int t = 0; t < NPAD; ++t) wv[t] *= cv[db * NPAD + t];  // W~_t = gamma_{n-1,t} w_t
+            // W~ split hi | lo into tensor memory, lane = value channel, column = token: the A of step 4
+            {
+                uint32_t hv[NPAD], lv[NPAD];
+#pragma unroll
+                for (int t = 0; t < NPAD; ++t) {
+                    const float hi = tf32_hi(wv[t]);
+                    hv[t] = __float_as_uint(hi);
+                    lv[t] = __float_as_uint(wv[t] - hi);
+                }
+                tmem_st16(tlane + TM_W, hv);
+                tmem_st16(tlane + TM_W + NPAD, lv);
+                tmem_wait_st();
+            }
+            // P = S_n^T U = g (S_0^T U) + sum_t w~_t (K U^T)_t
             if (P != nullptr) {
                 float pp[RP];
 #pragma unroll
-                for (int m = 0; m < RP; ++m) pp[m] = g * xp[NPAD + m];
+                for (int m = 0; m < RP; ++m) pp[m] = g * (xd[NPAD + m] + xd[NPAD + RP + m]);
 #pragma unroll
                 for (int t = 0; t < NPAD; ++t)
                     if (t < n)
 #pragma unroll
-                        for (int m = 0; m < RP; ++m) pp[m] = fmaf(acc[t], kus[t * RP + m], pp[m]);
+                        for (int m = 0; m < RP; ++m) pp[m] = fmaf(wv[t], kus[(db * NPAD + t) * RP + m], pp[m]);
                 float *prow = P + ((size_t)head * 128 + row) * r;
                 if ((r & 3) == 0) {
 #pragma unroll
@@ -603,32 +656,36 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
                         if (m < r) prow[m] = pp[m];
                 }
             }
-            fence_proxy_async();  // W~ is read by the tensor core
+        } else if (warp == 4 && w + 1 < w_end) {  // meanwhile: the next head's decay table
+            decay_table(a_nx, b_nx, db ^ 1);
         }
+        tc_fence_before();
         __syncthreads();
         // ---- step 4: D^T = W~^T K (hi and lo passes), both operands in shared memory
         if (warp == 0) {
             tc_fence_after();
+            if (elect_one()) {
 #pragma unroll 1
-            for (int pass = 0; pass < 2; ++pass)
+                for (int pass = 0; pass < 2; ++pass)
 #pragma unroll 1
-                for (int kk = 0; kk < kc; ++kk) {
-                    const uint64_t ad = smem_desc_kmajor_sw128((pass ? wl_a : wh_a) + kk * 32);
-                    const uint64_t bd = smem_desc_mnmajor_sw128_32b(kbm_a + kk * 1024, npad * 128);
-                    if (elect_one()) mma_ss(tbase + TM_D, ad, bd, idx_c, pass | kk);
-                }
-            if (elect_one()) mma_commit(bar_c);
+                    for (int kk = 0; kk < kc; ++kk) {
+                        const uint64_t bd = smem_desc_mnmajor_sw128_32b(kbm_a + kk * 1024, NPAD * 128);
+                        mma_ts(tbase + TM_D2, tbase + TM_W + NPAD * pass + 8 * kk, bd, idx_4, pass | kk);
+                    }
+                mma_commit(bar_4);
+            }
             __syncwarp();
-            ok = mbar_wait(bar_c, ph);
+            ok = mbar_wait(bar_4, ph);
         }
         if (__syncthreads_or(!ok)) { failed = true; break; }
         tc_fence_after();
-        // ---- step 5: S_n = g S_0 + D, back into the stage for the TMA store
+        // ---- step 5: S_n = g S_0 + D, back into the stage (its step-1 reads are complete), then out by
+        // TMA tiled stores
 #pragma unroll
         for (int j2 = 0; j2 < 2; ++j2) {
             const int pnl = 2 * half + j2;
             uint32_t d[32];
-            tmem_ld32(tlane + TM_D + 32 * pnl, d);
+            tmem_ld32(tlane + TM_D2 + 32 * pnl, d);
             tmem_wait_ld();
 #pragma unroll
             for (int q = 0; q < 8; ++q)
@@ -639,19 +696,13 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
                                 fmaf(g, s0[32 * j2 + 4 * q + 3], __uint_as_float(d[4 * q + 3])));
         }
         tc_fence_before();
-        fence_proxy_async();  // the updated state, written by these threads, is read by the TMA store
-        __syncthreads();
+        fence_proxy_async();  // the new state, written by these threads, is read by the TMA store
+        __syncthreads();  // tensor memory and the operands are free for the next head
         if (warp == 1) {
             if (elect_one()) {
                 for (int p = 0; p < 4; ++p) tma_store_2d(&tmS, 32 * p, head * 128, stage + p * TC_PANEL);
                 bulk_commit();
-                if (ns == 1 && w + 1 < w_end) {  // one stage: refill it as soon as the store has read it
-                    bulk_wait_read_all();
-                    fence_proxy_async();
-                    issue_state(w + 1, 0);
-                }
             }
-            if (ns == 1 && w + 1 < w_end) note_state(w + 1, 0);
             __syncwarp();
         }
     }
@@ -659,7 +710,7 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
     if (failed) {  // count the give-up, then let what is in flight land (bounded)
         if (warp == 1) {
             if (elect_one()) atomicAdd(&g_update_tc_giveups, 1u);
-            for (int st = 0; st < ns; ++st)
+            for (int st = 0; st < TC_NS; ++st)
                 if (pend_s & (1u << st)) mbar_wait(bar_s + st, (par_s >> st) & 1);
             for (int i = 0; i < 2; ++i)
                 if (pend_t & (1u << i)) mbar_wait(bar_t + i, (par_t >> i) & 1);
@@ -670,7 +721,7 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
         }
     }
     if (warp == 1) {
-        if (elect_one()) bulk_wait_all();
+        if (elect_one()) bulk_wait_all();  // the last stores have landed before the kernel ends
         __syncwarp();
     }
     tc_fence_before();
@@ -702,21 +753,16 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
 int update_tc_giveups(bool reset, unsigned *count) { return read_counter(&g_update_tc_giveups, reset, count); }
 
 // The Gated DeltaNet window update on the tensor cores, where it applies: dk = dv = 128, fp32
-// state, bf16 keys (exact in TF32, so each product takes two passes), 1 <= n <= 16 tokens, and a
-// shared-memory layout with at least two state stages (r <= 16 at W <= 16).
+// state, bf16 keys and values (keys exact in TF32), 1 <= n <= 16 tokens, r <= 16.
 // Returns TC_NOT_APPLICABLE for other shapes (the caller then runs the CUDA-core kernel), else a
 // sketchssm_status.
 int launch_update_window_tc(const sketchssm_dims &d, void *S, float *P, const float *U, const void *k,
                             const void *v, const float *alpha, const float *beta, int n, cudaStream_t stream) {
     if (d.kind != SKSSM_GDN || d.dk != 128 || d.dv != 128 || d.state_dtype != SKSSM_F32) return TC_NOT_APPLICABLE;
-    if (d.qkv_dtype != SKSSM_BF16 || n < 1 || n > 16 || d.W > 32 || d.r > 32) return TC_NOT_APPLICABLE;
-    const int npad = 16;
-    const int rp = d.r <= 4 ? 4 : d.r <= 8 ? 8 : d.r <= 16 ? 16 : 32;
-    int ns = 0;  // state stages: at least two, so that the next head's state loads behind this one
-    for (int cand = 3; cand >= 2 && !ns; --cand)
-        if (tc_layout(cand, npad, rp, d.W).total <= TC_SMEM_LIMIT) ns = cand;
-    if (!ns) return TC_NOT_APPLICABLE;
-    const TcLayout L = tc_layout(ns, npad, rp, d.W);
+    if (d.qkv_dtype != SKSSM_BF16 || n < 1 || n > TC_NPAD || d.r > 16) return TC_NOT_APPLICABLE;
+    const int rp = d.r <= 4 ? 4 : d.r <= 8 ? 8 : 16;
+    const TcLayout L = tc_layout(rp);
+    if (L.total > TC_SMEM_LIMIT) return TC_NOT_APPLICABLE;
     const int NH = d.B * d.H;
 
     PFN_cuTensorMapEncodeTiled_v12000 enc = encode_tiled();
@@ -731,25 +777,22 @@ int launch_update_window_tc(const sketchssm_dims &d, void *S, float *P, const fl
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return SKSSM_ERR_CUDA;
 
-    auto run = [&](auto NPc, auto RPc) -> int {
-        constexpr int NP = decltype(NPc)::value, RP = decltype(RPc)::value;
-        auto kern = update_window_gdn_tc<NP, RP>;
+    auto run = [&](auto RPc) -> int {
+        constexpr int RP = decltype(RPc)::value;
+        auto kern = update_window_gdn_tc<RP>;
         if (allow_max_smem(reinterpret_cast<const void *>(kern)) != SKSSM_OK) return SKSSM_ERR_CUDA;
         int sms = 0;
         if (sm_count(&sms) != SKSSM_OK) return SKSSM_ERR_CUDA;
         const int grid = NH < sms ? NH : sms;
-        kern<<<grid, TC_THREADS, L.total, stream>>>(map, P, U, static_cast<const __nv_bfloat16 *>(k),
+        kern<<<grid, TC_THREADS, L.total, stream>>>(map, P, U,
+                                                    static_cast<const __nv_bfloat16 *>(k),
                                                     static_cast<const __nv_bfloat16 *>(v), alpha, beta, d.B, d.H, d.r,
-                                                    n, d.W, ns);
+                                                    n, d.W);
         return launch_status();
     };
-    auto by_r = [&](auto NPc) -> int {
-        if (rp == 4) return run(NPc, std::integral_constant<int, 4>());
-        if (rp == 8) return run(NPc, std::integral_constant<int, 8>());
-        if (rp == 16) return run(NPc, std::integral_constant<int, 16>());
-        return run(NPc, std::integral_constant<int, 32>());
-    };
-    return by_r(std::integral_constant<int, 16>());
+    if (rp == 4) return run(std::integral_constant<int, 4>());
+    if (rp == 8) return run(std::integral_constant<int, 8>());
+    return run(std::integral_constant<int, 16>());
 }
 
 }  // namespace skssm

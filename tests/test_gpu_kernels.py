@@ -58,7 +58,8 @@ CASES = [
     ("kda", 128, 128, 8, 16, torch.bfloat16, torch.bfloat16),
     ("gdn", 64, 64, 4, 8, torch.bfloat16, torch.float32),
     ("kda", 128, 128, 128, 64, torch.float32, torch.float32),  # largest layout: one CTA per head
-    ("gdn", 128, 128, 4, 24, torch.float32, torch.float32),    # tensor-core update, fp32 tokens
+    ("gdn", 128, 128, 4, 24, torch.float32, torch.float32),    # fp32 tokens: the CUDA-core update
+    ("gdn", 128, 128, 16, 13, torch.float32, torch.bfloat16),  # n = 13: the tensor-core update, r = 16
 ]
 
 

@@ -605,6 +605,16 @@ def measure_workload(cfg, dev, stream, clocks, barrier, steps, warmup, peak):
     if tc_update(cfg):
         kernels["update_window"]["path"] = ("tensor cores: chunked form, S_0^T [K; U] and the rank-n increment "
                                             "on tcgen05 (kind::tf32, split operands)")
+    elif cfg.kind == "kda" and cfg.r <= 8 and cfg.state_dtype == "f32" and cfg.qkv_dtype == "bf16" and W <= 16:
+        # the tensor-core form of the KDA update, an explicit alternative (not the default), same windows
+        St, Pt = S.clone(), P.clone()
+        g_tc = [capture_graph(lambda b=b: rs.sketchssm_update_window_tc(d, St, Pt, U, b.k, b.v, b.alpha, b.beta, W),
+                              stream) for b in bufs]
+        t_tc, _ = timed_windows([g_tc], steps, warmup, stream, clocks, barrier)
+        del g_tc, St, Pt
+        kernels["update_window_tc"] = kernel_entry(bm["update"], t_tc, steps, peak)
+        kernels["update_window_tc"]["note"] = ("sketchssm_update_window_tc for KDA: chunked form on tcgen05 with "
+                                               "split decayed keys (not the default: slower than update_window)")
     dominant = "update_window" if t_upd >= t_dec else "decode_step"
     value, value_f = tok_steps / t_s, tok_steps / t_f
     speedup = value / value_f

@@ -139,14 +139,16 @@ int sketchssm_update_window_read(const sketchssm_dims *dims, void *S, float *P, 
                                  int n_tokens, const void *q, float *o, void *stream);
 
 /*
- * sketchssm_update_window_tc -- sketchssm_update_window for Gated DeltaNet with the
+ * sketchssm_update_window_tc -- sketchssm_update_window for the delta rules with the
  * window's tokens applied in chunked (WY) form, both products on the tensor cores
  * (tcgen05.mma kind::tf32): [X | S_0^T U] = S_0^T [K; U] with the state split into
  * its TF32 part and remainder, and the rank-n state increment W~^T K with W~ split
- * the same way, so the result matches the recurrence to fp32 rounding (keys are
- * exact in TF32).  The state moves by TMA tiled copies.  Applies to SKSSM_GDN with
- * dk = dv = 128, fp32 state, bf16 q/k/v, 1 <= n_tokens <= 16 and r <= 16; other
- * sizes return SKSSM_ERR_DIMS.  sketchssm_update_window takes this path by itself
+ * the same way, so the result matches the recurrence to fp32 rounding (Gated
+ * DeltaNet keys are exact in TF32; KDA's keys carry the per-channel decay products
+ * and are split too).  The state moves by TMA tiled copies.  Applies to SKSSM_GDN
+ * (r <= 16) and SKSSM_KDA (r <= 8) with dk = dv = 128, fp32 state, bf16 q/k/v and
+ * 1 <= n_tokens <= 16; other sizes return SKSSM_ERR_DIMS.  For KDA it is an
+ * alternative, not the default: it measured slower than the CUDA-core kernel.  sketchssm_update_window takes this path by itself
  * for 12 <= n_tokens <= 16; this entry forces it for any n_tokens >= 1 (below 12
  * tokens the CUDA-core kernel is faster).
  * Arguments and other errors as sketchssm_update_window (n_tokens >= 1).

@@ -66,7 +66,7 @@ int sketchssm_update_window(const sketchssm_dims *d, void *S, float *P, const fl
     if (n_tokens < 0 || n_tokens > d->W) return SKSSM_ERR_RANGE;
     if (n_tokens > 0 && (rc = check_tokens(d, k, v, alpha, beta))) return rc;
     if (!aligned(S, 16) || !aligned(P, 16) || !aligned(U, 16)) return SKSSM_ERR_ALIGN;
-    if (n_tokens >= TC_MIN_TOKENS) {  // the tensor-core form where it applies and pays
+    if (n_tokens >= TC_MIN_TOKENS && d->kind == SKSSM_GDN) {  // the tensor-core form where it pays
         rc = launch_update_window_tc(*d, S, P, P ? U : nullptr, k, v, alpha, beta, n_tokens, (cudaStream_t)stream);
         if (rc != TC_NOT_APPLICABLE) return rc;
     }

@@ -53,9 +53,11 @@ int launch_update_window(const sketchssm_dims &d, void *S, float *P, const float
 // The Gated DeltaNet window update on the tensor cores (update_window_tc.cu) where it applies;
 // TC_NOT_APPLICABLE otherwise (the caller runs the CUDA-core kernel).
 constexpr int TC_NOT_APPLICABLE = 1;
-// Fewest tokens for which sketchssm_update_window takes the tensor-core form: its cost hardly
-// depends on n, while the CUDA-core kernel's grows with n (Gated DeltaNet, B = 256, H = 32,
-// r = 8: 229 against 266 us per launch at n = 8, 358 against 303 us at n = 16).
+// Fewest tokens for which sketchssm_update_window takes the tensor-core form (Gated DeltaNet): its
+// cost hardly depends on n, while the CUDA-core kernel's grows with n (B = 256, H = 32, r = 8: 229
+// against 266 us per launch at n = 8, 358 against 303 us at n = 16).  KDA stays on the CUDA cores:
+// its tensor-core form measured slower (B = 512, r = 8, n = 16: 1004 against 793 us), the per-
+// channel decay products and the decayed Gram costing more on the CUDA cores than the products save.
 constexpr int TC_MIN_TOKENS = 12;
 int launch_update_window_tc(const sketchssm_dims &d, void *S, float *P, const float *U, const void *k,
                             const void *v, const float *alpha, const float *beta, int n_tokens, cudaStream_t stream);

@@ -76,16 +76,21 @@ constexpr uint32_t TM_W = 384;   // W~^T hi (16 columns) then lo (16): A of step
 constexpr int TC_SMEM_LIMIT = 227 * 1024;
 
 __host__ __device__ inline int round_up(int x, int a) { return (x + a - 1) / a * a; }
-__host__ __device__ constexpr int tc_n1(int rp) { return (TC_NPAD + 2 * rp + 15) / 16 * 16; }
+// rows of B1: key rows (16; KDA: 16 hi + 16 lo of the decayed keys), then U hi and U lo (rp each)
+__host__ __device__ constexpr int tc_nk(bool kda) { return kda ? 2 * TC_NPAD : TC_NPAD; }
+__host__ __device__ constexpr int tc_n1(int rp, bool kda) { return (tc_nk(kda) + 2 * rp + 15) / 16 * 16; }
 
 // Shared-memory layout: byte offsets from the 1024-aligned base.
 struct TcLayout {
     int stages;     // TC_NS x 64 KB: state stages (TMA destination; A of step 1's first pass)
-    int b1;         // B of step 1: N1 rows [keys (16) | U hi (RP) | U lo (RP) | 0] x 128 fp32, K-major,
+    int b1;         // B of step 1: N1 rows [keys | U hi (RP) | U lo (RP) | 0] x 128 fp32, K-major,
                     // 128-byte swizzle, 4 panels of N1 rows x 128 B
-    int kbm;        // the keys, MN-major TF32 layout: 4 panels x 16 rows x 128 B (B of step 4)
-    int tok;        // two token buffers: 16 key rows then 16 value rows, bf16
+    int kbm;        // the keys of step 4, MN-major TF32 layout: 4 panels x 16 rows x 128 B (KDA: the
+                    // decayed keys, hi then lo)
+    int tok;        // two token buffers: 16 key rows, 16 value rows (bf16), KDA: 16 decay rows (fp32)
     int tok_bytes;  // bytes of one token buffer
+    int uf;         // KDA: the basis rows of the current head index, fp32 [RP][128]
+    int gnv;        // KDA: the window's decay product per key channel, fp32 [128]
     int am;         // by head parity: A, decay table [2][16][20] each, K U^T [2][16][RP], b_t g_t,
                     // gamma_{n-1,t}, b_t [2][16] each, g [2]
     int bars;       // mbarriers: 2 stages, 2 token buffers, step 1, step 4, drain
@@ -93,15 +98,17 @@ struct TcLayout {
     int total;      // bytes to request (with slack for aligning the base)
 };
 
-__host__ __device__ inline TcLayout tc_layout(int rp) {
+__host__ __device__ inline TcLayout tc_layout(int rp, bool kda) {
     TcLayout L;
-    const int n1 = tc_n1(rp);
+    const int n1 = tc_n1(rp, kda);
     int o = 0;
     L.stages = o; o += TC_NS * TC_STATE;
     L.b1 = o; o += round_up(n1 * 512, 1024);
-    L.kbm = o; o += TC_NPAD * 512;
-    L.tok_bytes = 2 * TC_NPAD * 128 * 2;
+    L.kbm = o; o += (kda ? 2 : 1) * TC_NPAD * 512;
+    L.tok_bytes = 2 * TC_NPAD * 128 * 2 + (kda ? TC_NPAD * 128 * 4 : 0);
     L.tok = o; o += 2 * L.tok_bytes;
+    L.uf = o; o += kda ? rp * 512 : 0;
+    L.gnv = o; o += kda ? 512 : 0;
     L.am = o; o += round_up((4 * TC_NPAD * (TC_NPAD + 4) + 2 * TC_NPAD * rp + 6 * TC_NPAD + 4) * 4, 16);
     L.bars = o; o += 8 * (TC_NS + 5);
     L.slot = o; o += 16;
@@ -278,18 +285,19 @@ __device__ __forceinline__ float dot4(float4 a, float4 b) {
     return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, a.w * b.w)));
 }
 
-template <int RP>
+template <int KIND, int RP>
 __global__ void __launch_bounds__(TC_THREADS, 1)
-update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict__ P,
+update_window_delta_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict__ P,
                      const float *__restrict__ U, const __nv_bfloat16 *__restrict__ kbuf,
                      const __nv_bfloat16 *__restrict__ vbuf, const float *__restrict__ abuf,
                      const float *__restrict__ bbuf, int B, int H, int r, int n, int W) {
     using QT = __nv_bfloat16;
-    constexpr int NPAD = TC_NPAD, N1 = tc_n1(RP), as = NPAD + 4;  // rows of A and G: 16-byte aligned
+    constexpr bool KD = KIND == KDA;
+    constexpr int NPAD = TC_NPAD, NK = tc_nk(KD), N1 = tc_n1(RP, KD), as = NPAD + 4;  // A, G rows: 16-B aligned
     constexpr int B1P = N1 * 128;  // bytes of one 32-column panel of B1
     extern __shared__ __align__(1024) unsigned char tc_raw[];
     unsigned char *sm = tc_raw + ((1024 - (smem_u32(tc_raw) & 1023)) & 1023);
-    const TcLayout L = tc_layout(RP);
+    const TcLayout L = tc_layout(RP, KD);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int quad = warp & 3, half = warp >> 2;
     const int row = 32 * quad + lane;  // this thread's state row (value channel) and tensor-memory lane
@@ -305,8 +313,9 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
     uint64_t *bar_d = bar_4 + 1;                                  // the drain after a give-up
     uint32_t *slot = reinterpret_cast<uint32_t *>(sm + L.slot);
     // per head parity:
-    float *Am = reinterpret_cast<float *>(sm + L.am);  // [2][16][as]: A[t][s] = b_t gamma_{t,s} G[t][s] (s < t, else 0)
-    float *Gam = Am + 2 * NPAD * as;                    // [2][16][as]: b_t gamma_{t,s} (s < t, else 0)
+    // A[t][s] = b_t gamma_{t,s} G[t][s] (GDN) or b_t sum_i gamma_{t,s,i} k_t,i k_s,i (KDA), s < t; else 0
+    float *Am = reinterpret_cast<float *>(sm + L.am);  // [2][16][as]
+    float *Gam = Am + 2 * NPAD * as;                    // [2][16][as]: b_t gamma_{t,s} (KDA: b_t), s < t; else 0
     float *kus = Gam + 2 * NPAD * as;                   // [2][16][RP]: (K U^T)[t][m]
     float *ev = kus + 2 * NPAD * RP;                    // [2][16]: b_t g_t
     float *cv = ev + 2 * NPAD;                          // [2][16]: gamma_{n-1,s}
@@ -314,7 +323,10 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
     float *gn = bv + 2 * NPAD;                          // [2]:  g_{n-1}
     unsigned char *b1 = sm + L.b1, *kbm = sm + L.kbm;
     const uint32_t b1_a = smem_u32(b1), kbm_a = smem_u32(kbm);
+    float *uf = reinterpret_cast<float *>(sm + L.uf);    // KDA: [RP][128] basis rows of the current h
+    float *gnv = reinterpret_cast<float *>(sm + L.gnv);  // KDA: [128] the window's decay product g_{n-1}
     const int kbytes = n * 128 * (int)sizeof(QT);
+    constexpr int AOFF = 2 * NPAD * 128 * (int)sizeof(QT);  // KDA: decay rows after the keys and values
 
     auto head_of = [&](int w) { return (w % B) * H + w / B; };
     auto stage_of = [&](int st) { return sm + L.stages + st * TC_STATE; };
@@ -328,9 +340,10 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
     auto issue_tok = [&](int w, int i) {
         uint64_t *bar = bar_t + i;
         const size_t off = (size_t)head_of(w) * W * 128;
-        mbar_expect_tx(bar, 2 * kbytes);
+        mbar_expect_tx(bar, 2 * kbytes + (KD ? n * 512 : 0));
         bulk_g2s(tok_of(i), kbuf + off, kbytes, bar);
         bulk_g2s(tok_of(i) + NPAD * 128 * sizeof(QT), vbuf + off, kbytes, bar);
+        if (KD) bulk_g2s(tok_of(i) + AOFF, abuf + off, n * 512, bar);
     };
 
     float a_nx = 1.f, b_nx = 0.f;  // warp 4, lane t: a_t and b_t of the next head to build a system for
@@ -368,9 +381,70 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
     };
 
     // warps 2, 3, 6, 7 (not the sub-partitions of the MMA and copy issuers): this head's key Gram and
-    // K U^T from the fp32 rows of B1 (keys, U hi and lo), and A = (b_t gamma_{t,s}) o G into buffer buf
-    auto gram_system = [&](int buf) {
+    // K U^T, and A = (b_t gamma_{t,s}) o G into buffer buf.  GDN: from the fp32 rows of B1 (keys, U hi
+    // and lo).  KDA: from the token buffer tk (keys, per-channel decays) and the basis rows uf, with
+    // the channel decays between the two tokens inside the dot.
+    auto gram_system = [&](int buf, const unsigned char *tk) {
         const int t0 = 4 * ((warp & 1) + (warp >> 1 & 2));  // rows t0 .. t0 + 3
+        if constexpr (KD) {
+            const QT *kr = reinterpret_cast<const QT *>(tk);
+            const float *ar = reinterpret_cast<const float *>(tk + AOFF);
+            auto krow = [&](int t) {  // key channels 4 lane .. + 3 of token t (zero past n)
+                float f[4] = {0.f, 0.f, 0.f, 0.f};
+                if (t < n) load4(kr + t * 128 + 4 * lane, f);
+                return make_float4(f[0], f[1], f[2], f[3]);
+            };
+            auto arow = [&](int t) { return *reinterpret_cast<const float4 *>(ar + t * 128 + 4 * lane); };
+            auto mul4 = [](float4 a, float4 b) { return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w); };
+            float4 ks[NPAD];
+#pragma unroll
+            for (int j = 0; j < NPAD; ++j) ks[j] = krow(j);
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {  // rows t0 + 2g, t0 + 2g + 1: sum_i gamma_{t,s,i} k_t,i k_s,i, s < t
+                float v[32];
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr) {
+                    const int t = t0 + 2 * g + rr;
+                    const float4 kt_ = krow(t);
+                    float4 gm = make_float4(1.f, 1.f, 1.f, 1.f);
+#pragma unroll
+                    for (int s2 = NPAD - 1; s2 >= 0; --s2) {
+                        if (s2 < t && t < n) {
+                            gm = mul4(gm, arow(s2 + 1));  // gamma_{t,s} = a_{s+1} ... a_t
+                            v[16 * rr + s2] = dot4(mul4(kt_, gm), ks[s2]);
+                        } else {
+                            v[16 * rr + s2] = 0.f;
+                        }
+                    }
+                }
+                warp_reduce_scatter32(v, lane);
+                const int tt = t0 + 2 * g + (lane >> 4), ss = lane & 15;
+                Am[(buf * NPAD + tt) * as + ss] = Gam[(buf * NPAD + tt) * as + ss] * v[0];
+            }
+            float4 kk[4];  // gamma_{n-1,t} o k_t for the warp's rows
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int t = t0 + j;
+                float4 gm = make_float4(1.f, 1.f, 1.f, 1.f);
+                for (int u = t + 1; u < n; ++u) gm = mul4(gm, arow(u));
+                kk[j] = mul4(krow(t), gm);
+            }
+#pragma unroll
+            for (int m0 = 0; m0 < RP; m0 += 8) {  // (gamma_{n-1,t} o k_t) . U_m
+                float4 uu[8];
+#pragma unroll
+                for (int m = 0; m < 8; ++m)
+                    uu[m] = m0 + m < RP ? *reinterpret_cast<const float4 *>(uf + (m0 + m) * 128 + 4 * lane)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                float v[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = dot4(kk[i >> 3], uu[i & 7]);
+                warp_reduce_scatter32(v, lane);
+                const int m = m0 + (lane & 7);
+                if (m < RP) kus[(buf * NPAD + t0 + (lane >> 3)) * RP + m] = v[0];
+            }
+            return;
+        }
         // lane l: key channels 4l .. 4l+3 (panel l / 8, chunk l % 8 of its 128-byte rows)
         const unsigned char *pn = b1 + (lane >> 3) * B1P;
         auto rowv = [&](int rr) {
@@ -397,7 +471,7 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
 #pragma unroll
             for (int m = 0; m < 8; ++m) {
                 if (m0 + m < RP) {
-                    const float4 uh = rowv(NPAD + m0 + m), ul = rowv(NPAD + RP + m0 + m);
+                    const float4 uh = rowv(NK + m0 + m), ul = rowv(NK + RP + m0 + m);
                     uu[m] = make_float4(uh.x + ul.x, uh.y + ul.y, uh.z + ul.z, uh.w + ul.w);
                 } else {
                     uu[m] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -423,8 +497,10 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    // the key rows n .. 15 of B1 and of the MN-major keys stay zero for the whole run
-    for (int i = tid; i < (4 * B1P + NPAD * 512) / 16; i += TC_THREADS) {
+    // the key rows n .. 15 of B1 and of the MN-major keys stay zero for the whole run (GDN; KDA rewrites
+    // them every head), and so do B1's padding rows
+    constexpr int KBM_BYTES = (KD ? 2 : 1) * NPAD * 512;
+    for (int i = tid; i < (4 * B1P + KBM_BYTES) / 16; i += TC_THREADS) {
         unsigned char *dst = i < 4 * B1P / 16 ? b1 + 16 * i : kbm + 16 * (i - 4 * B1P / 16);
         *reinterpret_cast<float4 *>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
@@ -455,9 +531,9 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
         __syncwarp();
     }
     // per-token scalars, prefetched one head ahead by warp 4 (lane t holds token t)
-    if (warp == 4) {
+    if (warp == 4) {  // (KDA: the decays are per channel and enter elsewhere; its table keeps a = 1)
         if (lane < n) {
-            a_nx = abuf[(size_t)head_of(w_begin) * W + lane];
+            if (!KD) a_nx = abuf[(size_t)head_of(w_begin) * W + lane];
             b_nx = bbuf[(size_t)head_of(w_begin) * W + lane];
         }
         decay_table(a_nx, b_nx, 0);  // the first head's
@@ -482,14 +558,19 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
         }
         const int db = it & 1;  // this head's decay table
         if (warp == 4 && w + 1 < w_end && lane < n) {  // the next head's scalars, for its table
-            a_nx = abuf[(size_t)head_of(w + 1) * W + lane];
+            if (!KD) a_nx = abuf[(size_t)head_of(w + 1) * W + lane];
             b_nx = bbuf[(size_t)head_of(w + 1) * W + lane];
         }
-        if (h != h_prev) {  // basis rows of head index h into B1 rows 16 .. (hi, then lo; rows past r zero)
+        if (h != h_prev) {  // basis rows of head index h (rows past r zero): GDN into B1 rows 16 .. (hi, then
+                            // lo); KDA into uf (B1's rows are scaled by each head's decay product)
             for (int i = tid; i < RP * 32; i += TC_THREADS) {
                 const int m = i >> 5, c4 = (i & 31) * 4;
                 float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (P != nullptr && m < r) u = reinterpret_cast<const float4 *>(U + ((size_t)h * r + m) * 128)[i & 31];
+                if (KD) {
+                    reinterpret_cast<float4 *>(uf)[i] = u;
+                    continue;
+                }
                 const float4 uh = make_float4(tf32_hi(u.x), tf32_hi(u.y), tf32_hi(u.z), tf32_hi(u.w));
                 const float4 ul = make_float4(u.x - uh.x, u.y - uh.y, u.z - uh.z, u.w - uh.w);
                 unsigned char *pn = b1 + (c4 >> 5) * B1P;
@@ -510,6 +591,51 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
         }
         if (__syncthreads_or(!ok)) { failed = true; break; }
         // ---- the keys as fp32 rows of B1 (K-major) and of the MN-major operand of step 4
+        if constexpr (KD) {
+            // per key channel i: threads 0-127 the prefix products g_t (keys of step 1: g_t o k_t,
+            // hi and lo; the basis rows g_{n-1} o U_m, hi and lo; g_{n-1} for the store), threads
+            // 128-255 the suffix products gamma_{n-1,s} (keys of step 4, hi and lo)
+            const int i = tid & 127, ci = i & 31;
+            const QT *kr = reinterpret_cast<const QT *>(tk);
+            const float *ar = reinterpret_cast<const float *>(tk + AOFF);
+            if (tid < 128) {
+                unsigned char *pn = b1 + (i >> 5) * B1P;
+                float g = 1.f;
+#pragma unroll
+                for (int t = 0; t < NPAD; ++t) {
+                    float kg = 0.f;
+                    if (t < n) {
+                        g *= ar[t * 128 + i];
+                        kg = g * ld1(kr + t * 128 + i);
+                    }
+                    const float hi = tf32_hi(kg);
+                    *reinterpret_cast<float *>(pn + sw128(t, ci)) = hi;
+                    *reinterpret_cast<float *>(pn + sw128(NPAD + t, ci)) = kg - hi;
+                }
+                gnv[i] = g;
+#pragma unroll
+                for (int m = 0; m < RP; ++m) {
+                    const float ug = g * uf[m * 128 + i];
+                    const float hi = tf32_hi(ug);
+                    *reinterpret_cast<float *>(pn + sw128(NK + m, ci)) = hi;
+                    *reinterpret_cast<float *>(pn + sw128(NK + RP + m, ci)) = ug - hi;
+                }
+            } else {
+                unsigned char *dh = kbm + (i >> 5) * (NPAD * 128), *dl = dh + NPAD * 512;
+                float gam = 1.f;  // gamma_{n-1,s} = a_{s+1} ... a_{n-1}, s descending
+#pragma unroll
+                for (int s2 = NPAD - 1; s2 >= 0; --s2) {
+                    float kk = 0.f;
+                    if (s2 < n) {
+                        kk = gam * ld1(kr + s2 * 128 + i);
+                        gam *= ar[s2 * 128 + i];
+                    }
+                    const float hi = tf32_hi(kk);
+                    *reinterpret_cast<float *>(dh + sw128_32b(s2, ci)) = hi;
+                    *reinterpret_cast<float *>(dl + sw128_32b(s2, ci)) = kk - hi;
+                }
+            }
+        } else
         for (int i = tid; i < n * 16; i += TC_THREADS) {
             const int t = i >> 4, c8 = (i & 15) * 8;
             float x[8];
@@ -575,7 +701,7 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
             }
             __syncwarp();
         } else if ((warp & 2) != 0) {  // ---- step 2 under step 1
-            gram_system(db);
+            gram_system(db, tk);
         }
         // ---- step 1 complete
         if (warp == 0) ok = mbar_wait(bar_1, ph);
@@ -608,7 +734,9 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
 #pragma unroll
             for (int t = 0; t < NPAD; ++t) {  // (I + A) w = y, forward (A[t][s] = 0 for s >= t)
                 // (value rows past n are not copied: their shared memory is not read)
-                float y0 = t < n ? bv[db * NPAD + t] * ld1(vt + t * 128 + row) - ev[db * NPAD + t] * xd[t] : 0.f,
+                // x_t = S_0^T k_t (KDA: S_0^T (g_t o k_t), from its hi and lo key rows)
+                const float xt = KD ? xd[t] + xd[NPAD + t] : xd[t];
+                float y0 = t < n ? bv[db * NPAD + t] * ld1(vt + t * 128 + row) - ev[db * NPAD + t] * xt : 0.f,
                       y1 = 0.f;
 #pragma unroll
                 for (int s4 = 0; s4 < t; s4 += 4) {
@@ -639,7 +767,7 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
             if (P != nullptr) {
                 float pp[RP];
 #pragma unroll
-                for (int m = 0; m < RP; ++m) pp[m] = g * (xd[NPAD + m] + xd[NPAD + RP + m]);
+                for (int m = 0; m < RP; ++m) pp[m] = g * (xd[NK + m] + xd[NK + RP + m]);
 #pragma unroll
                 for (int t = 0; t < NPAD; ++t)
                     if (t < n)
@@ -661,16 +789,17 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
         }
         tc_fence_before();
         __syncthreads();
-        // ---- step 4: D^T = W~^T K (hi and lo passes), both operands in shared memory
+        // ---- step 4: D^T = W~^T K (W~ hi and lo passes; KDA: also W~ hi against the decayed keys' lo)
         if (warp == 0) {
             tc_fence_after();
             if (elect_one()) {
 #pragma unroll 1
-                for (int pass = 0; pass < 2; ++pass)
+                for (int pass = 0; pass < (KD ? 3 : 2); ++pass)
 #pragma unroll 1
                     for (int kk = 0; kk < kc; ++kk) {
-                        const uint64_t bd = smem_desc_mnmajor_sw128_32b(kbm_a + kk * 1024, NPAD * 128);
-                        mma_ts(tbase + TM_D2, tbase + TM_W + NPAD * pass + 8 * kk, bd, idx_4, pass | kk);
+                        const uint64_t bd = smem_desc_mnmajor_sw128_32b(
+                            kbm_a + (pass == 2 ? NPAD * 512 : 0) + kk * 1024, NPAD * 128);
+                        mma_ts(tbase + TM_D2, tbase + TM_W + (pass == 1 ? NPAD : 0) + 8 * kk, bd, idx_4, pass | kk);
                     }
                 mma_commit(bar_4);
             }
@@ -679,8 +808,8 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
         }
         if (__syncthreads_or(!ok)) { failed = true; break; }
         tc_fence_after();
-        // ---- step 5: S_n = g S_0 + D, back into the stage (its step-1 reads are complete), then out by
-        // TMA tiled stores
+        // ---- step 5: S_n = g S_0 + D (KDA: g per key channel), back into the stage (its step-1 reads are
+        // complete), then out by TMA tiled stores
 #pragma unroll
         for (int j2 = 0; j2 < 2; ++j2) {
             const int pnl = 2 * half + j2;
@@ -688,12 +817,14 @@ update_window_gdn_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict_
             tmem_ld32(tlane + TM_D2 + 32 * pnl, d);
             tmem_wait_ld();
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
+            for (int q = 0; q < 8; ++q) {
+                const float4 g4 = KD ? *reinterpret_cast<const float4 *>(gnv + 32 * pnl + 4 * q) : make_float4(g, g, g, g);
                 *reinterpret_cast<float4 *>(stage + pnl * TC_PANEL + sw128(row, 4 * q)) =
-                    make_float4(fmaf(g, s0[32 * j2 + 4 * q], __uint_as_float(d[4 * q])),
-                                fmaf(g, s0[32 * j2 + 4 * q + 1], __uint_as_float(d[4 * q + 1])),
-                                fmaf(g, s0[32 * j2 + 4 * q + 2], __uint_as_float(d[4 * q + 2])),
-                                fmaf(g, s0[32 * j2 + 4 * q + 3], __uint_as_float(d[4 * q + 3])));
+                    make_float4(fmaf(g4.x, s0[32 * j2 + 4 * q], __uint_as_float(d[4 * q])),
+                                fmaf(g4.y, s0[32 * j2 + 4 * q + 1], __uint_as_float(d[4 * q + 1])),
+                                fmaf(g4.z, s0[32 * j2 + 4 * q + 2], __uint_as_float(d[4 * q + 2])),
+                                fmaf(g4.w, s0[32 * j2 + 4 * q + 3], __uint_as_float(d[4 * q + 3])));
+            }
         }
         tc_fence_before();
         fence_proxy_async();  // the new state, written by these threads, is read by the TMA store
@@ -752,16 +883,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
 
 int update_tc_giveups(bool reset, unsigned *count) { return read_counter(&g_update_tc_giveups, reset, count); }
 
-// The Gated DeltaNet window update on the tensor cores, where it applies: dk = dv = 128, fp32
-// state, bf16 keys and values (keys exact in TF32), 1 <= n <= 16 tokens, r <= 16.
+// The delta-rule window update on the tensor cores, where it applies: Gated DeltaNet or KDA,
+// dk = dv = 128, fp32 state, bf16 keys and values (keys exact in TF32), 1 <= n <= 16 tokens,
+// r <= 16 (KDA: r <= 8, whose split decayed keys and basis rows take more shared memory).
 // Returns TC_NOT_APPLICABLE for other shapes (the caller then runs the CUDA-core kernel), else a
 // sketchssm_status.
 int launch_update_window_tc(const sketchssm_dims &d, void *S, float *P, const float *U, const void *k,
                             const void *v, const float *alpha, const float *beta, int n, cudaStream_t stream) {
-    if (d.kind != SKSSM_GDN || d.dk != 128 || d.dv != 128 || d.state_dtype != SKSSM_F32) return TC_NOT_APPLICABLE;
-    if (d.qkv_dtype != SKSSM_BF16 || n < 1 || n > TC_NPAD || d.r > 16) return TC_NOT_APPLICABLE;
+    const bool kda = d.kind == SKSSM_KDA;
+    if ((d.kind != SKSSM_GDN && !kda) || d.dk != 128 || d.dv != 128 || d.state_dtype != SKSSM_F32)
+        return TC_NOT_APPLICABLE;
+    if (d.qkv_dtype != SKSSM_BF16 || n < 1 || n > TC_NPAD || d.r > (kda ? 8 : 16)) return TC_NOT_APPLICABLE;
     const int rp = d.r <= 4 ? 4 : d.r <= 8 ? 8 : 16;
-    const TcLayout L = tc_layout(rp);
+    const TcLayout L = tc_layout(rp, kda);
     if (L.total > TC_SMEM_LIMIT) return TC_NOT_APPLICABLE;
     const int NH = d.B * d.H;
 
@@ -777,22 +911,24 @@ int launch_update_window_tc(const sketchssm_dims &d, void *S, float *P, const fl
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return SKSSM_ERR_CUDA;
 
-    auto run = [&](auto RPc) -> int {
-        constexpr int RP = decltype(RPc)::value;
-        auto kern = update_window_gdn_tc<RP>;
+    auto run = [&](auto KINDc, auto RPc) -> int {
+        constexpr int KIND = decltype(KINDc)::value, RP = decltype(RPc)::value;
+        auto kern = update_window_delta_tc<KIND, RP>;
         if (allow_max_smem(reinterpret_cast<const void *>(kern)) != SKSSM_OK) return SKSSM_ERR_CUDA;
         int sms = 0;
         if (sm_count(&sms) != SKSSM_OK) return SKSSM_ERR_CUDA;
         const int grid = NH < sms ? NH : sms;
-        kern<<<grid, TC_THREADS, L.total, stream>>>(map, P, U,
-                                                    static_cast<const __nv_bfloat16 *>(k),
+        kern<<<grid, TC_THREADS, L.total, stream>>>(map, P, U, static_cast<const __nv_bfloat16 *>(k),
                                                     static_cast<const __nv_bfloat16 *>(v), alpha, beta, d.B, d.H, d.r,
                                                     n, d.W);
         return launch_status();
     };
-    if (rp == 4) return run(std::integral_constant<int, 4>());
-    if (rp == 8) return run(std::integral_constant<int, 8>());
-    return run(std::integral_constant<int, 16>());
+    using G = std::integral_constant<int, GDN>;
+    using K = std::integral_constant<int, KDA>;
+    if (kda) return rp == 4 ? run(K(), std::integral_constant<int, 4>()) : run(K(), std::integral_constant<int, 8>());
+    if (rp == 4) return run(G(), std::integral_constant<int, 4>());
+    if (rp == 8) return run(G(), std::integral_constant<int, 8>());
+    return run(G(), std::integral_constant<int, 16>());
 }
 
 }  // namespace skssm

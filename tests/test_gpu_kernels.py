@@ -244,19 +244,20 @@ def test_update_window_many_heads_per_cta(kind):
         assert state_err(P.reshape(B * H, dv, r).double().cpu().numpy(), Pref) <= STATE_TOL, n
 
 
-TC_PIPE = [(16, 8), (16, 13), (8, 4), (16, 16), (4, 1)]
+TC_PIPE = [("gdn", 16, 8), ("gdn", 16, 13), ("gdn", 8, 4), ("gdn", 16, 16), ("gdn", 4, 1),
+           ("kda", 16, 8), ("kda", 16, 3), ("kda", 8, 4)]
 
 
-@pytest.mark.parametrize("case", TC_PIPE, ids=[f"W{c[0]}-r{c[1]}" for c in TC_PIPE])
+@pytest.mark.parametrize("case", TC_PIPE, ids=[f"{c[0]}-W{c[1]}-r{c[2]}" for c in TC_PIPE])
 def test_update_window_tc_pipeline(case):
-    """sketchssm_update_window_tc, the Gated DeltaNet update with the state increment on the tensor
-    cores (dk = dv = 128, fp32 state, bf16 keys), over 2100 heads (B=7, H=300): each persistent CTA
-    runs ~15 heads through its state stages, reusing stages, token buffers and barrier phases,
-    across changes of h; full and partial windows, ranks that need padding.  Every head is checked."""
+    """sketchssm_update_window_tc, the delta-rule update on the tensor cores (dk = dv = 128, fp32
+    state, bf16 keys), over 2100 heads (B=7, H=300): each persistent CTA runs ~15 heads through its
+    state stages, reusing stages, token buffers and barrier phases, across changes of h; full and
+    partial windows, ranks that need padding.  Every head is checked."""
     import recurrent_state_read_b200 as rs
 
-    W, r = case
-    cfg, d, S0, U, R, tok = _setup("gdn", 128, 128, r, W, torch.float32, torch.bfloat16, B=7, H=300, seed=11)
+    kind, W, r = case
+    cfg, d, S0, U, R, tok = _setup(kind, 128, 128, r, W, torch.float32, torch.bfloat16, B=7, H=300, seed=11)
     B, H = d.B, d.H
     Uh = oracle.per_head(U, H, np.arange(B * H))
     ft = flat_tokens(tok)
@@ -269,7 +270,7 @@ def test_update_window_tc_pipeline(case):
         rs.sketchssm_update_window_tc(d, S, P, Ug, dev["k"], dev["v"], dev["alpha"], dev["beta"], n)
         torch.cuda.synchronize()
         sl = slice(0, n)
-        Sref, Pref = oracle.update_window("gdn", S0, Uh, ft["k"][sl], ft["v"][sl], ft["alpha"][sl], ft["beta"][sl])
+        Sref, Pref = oracle.update_window(kind, S0, Uh, ft["k"][sl], ft["v"][sl], ft["alpha"][sl], ft["beta"][sl])
         es = state_err(to_logical(S), Sref)
         ep = state_err(P.reshape(B * H, 128, r).double().cpu().numpy(), Pref)
         assert es <= STATE_TOL and ep <= STATE_TOL, (n, es, ep)
@@ -479,10 +480,10 @@ def test_update_window_tc_not_applicable():
     """Sizes outside the tensor-core update's envelope are rejected before any launch."""
     import recurrent_state_read_b200 as rs
 
-    cfg, d, S0, U, R, tok = _setup("kda", 128, 128, 8, 16, torch.float32, torch.bfloat16)
+    cfg, d, S0, U, R, tok = _setup("kda", 128, 128, 16, 16, torch.float32, torch.bfloat16)  # KDA: r <= 8
     dev = to_window(to_device(tok))
     S = to_gpu_state(S0, d.B, d.H)
-    P = torch.zeros(d.B, d.H, 128, 8, device="cuda")
+    P = torch.zeros(d.B, d.H, 128, 16, device="cuda")
     with pytest.raises(rs.SketchSSMError):
         rs.sketchssm_update_window_tc(d, S, P, U.transpose(1, 2).contiguous().cuda(), dev["k"], dev["v"],
                                       dev["alpha"], dev["beta"], 16)

@@ -1,4 +1,4 @@
-// update_window_tc.cu -- the Gated DeltaNet window update on the tensor cores.
+// update_window_tc.cu -- the delta-rule window update (Gated DeltaNet, KDA) on the tensor cores.
 //
 // SketchSSM (arXiv 2609.33051v1), Abstract: once per window the full state is
 // read, the buffered tokens are applied exactly and the basis outputs are
@@ -28,8 +28,9 @@
 // significant bits of an fp32 value: the tensor core drops the 13 low mantissa
 // bits (measured: 1 + 0.75 ulp of TF32 enters as 1).  The state goes in as it
 // arrived (the tensor core takes its TF32 part t(S_0)) and as its remainder
-// S_0 - t(S_0), exact in fp32, of which the tensor core keeps the top 11 bits; the keys are bf16, exact
-// in TF32; the basis rows go in split as U = hi + lo with hi exactly TF32.  So
+// S_0 - t(S_0), exact in fp32, of which the tensor core keeps the top 11 bits;
+// Gated DeltaNet's keys are bf16, exact in TF32; the basis rows go in split as
+// U = hi + lo with hi exactly TF32.  So
 // every product of step 1 is off by less than 2^-21 of its terms.  W~ is split
 // the same way for step 4.
 //
@@ -48,6 +49,12 @@
 // (off the issuers' sub-partitions); warps 0-3 (one value channel per thread)
 // solve, while warp 4 builds the next head's decay products.  Tensor memory (512
 // columns): the remainder (128), [X | S_0^T U] (<= 128), D (128), W~ hi | lo (32).
+// KDA (decay per key channel i, S_t = (I - b_t k_t k_t^T) diag(a_t) S_{t-1} + b_t k_t v_t^T): the
+// same steps with g_t, gamma_{t,s} per channel, x_t = S_0^T (g_t o k_t), A[t][s] = b_t
+// sum_i gamma_{t,s,i} k_t,i k_s,i, W~ = w, the keys of step 4 gamma_{n-1,s} o k_s, the basis rows
+// of step 1 g_{n-1} o U, and the store S_n = g_{n-1} o S_0 + D per key channel.  Those keys and
+// rows are fp32, so they are split hi + lo too (step 4 takes a third pass: W~ hi against the keys'
+// lo).  Per-channel prefix and suffix products are formed by one thread per channel.
 // Every wait is bounded; a wait that gives up is counted
 // (sketchssm_device_error_count), the CTA drains what it has in flight (bounded),
 // frees its tensor memory and returns.

@@ -84,6 +84,10 @@ int sketchssm_update_window_read(const sketchssm_dims *d, void *S, float *P, con
     if (n_tokens > 0 && (rc = check_tokens(d, k, v, alpha, beta))) return rc;
     if (!aligned(S, 16) || !aligned(P, 16) || !aligned(U, 16) || !aligned(q, 16) || !aligned(o, 16))
         return SKSSM_ERR_ALIGN;
+    if (n_tokens >= TC_MIN_TOKENS && d->kind == SKSSM_GDN) {  // the tensor-core form where it pays
+        rc = launch_update_window_tc(*d, S, P, U, k, v, alpha, beta, n_tokens, (cudaStream_t)stream, q, o);
+        if (rc != TC_NOT_APPLICABLE) return rc;
+    }
     return launch_update_window(*d, S, P, U, k, v, alpha, beta, n_tokens, q, o, nullptr, 0, 0, nullptr,
                                 (cudaStream_t)stream);
 }

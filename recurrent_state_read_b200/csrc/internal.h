@@ -60,7 +60,8 @@ constexpr int TC_NOT_APPLICABLE = 1;
 // channel decay products and the decayed Gram costing more on the CUDA cores than the products save.
 constexpr int TC_MIN_TOKENS = 12;
 int launch_update_window_tc(const sketchssm_dims &d, void *S, float *P, const float *U, const void *k,
-                            const void *v, const float *alpha, const float *beta, int n_tokens, cudaStream_t stream);
+                            const void *v, const float *alpha, const float *beta, int n_tokens, cudaStream_t stream, const void *q = nullptr,
+                            float *o = nullptr);
 // Counts of bounded in-kernel waits that gave up (window update, decode step); reset clears them.
 int update_wait_giveups(bool reset, unsigned *count);
 int update_tc_giveups(bool reset, unsigned *count);

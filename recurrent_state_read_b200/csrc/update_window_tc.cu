@@ -98,6 +98,7 @@ struct TcLayout {
     int tok_bytes;  // bytes of one token buffer
     int uf;         // KDA: the basis rows of the current head index, fp32 [RP][128]
     int gnv;        // KDA: the window's decay product per key channel, fp32 [128]
+    int xo;         // the exact read's partial sums of the second column half, fp32 [128]
     int am;         // by head parity: A, decay table [2][16][20] each, K U^T [2][16][RP], b_t g_t,
                     // gamma_{n-1,t}, b_t [2][16] each, g [2]
     int bars;       // mbarriers: 2 stages, 2 token buffers, step 1, step 4, drain
@@ -116,6 +117,7 @@ __host__ __device__ inline TcLayout tc_layout(int rp, bool kda) {
     L.tok = o; o += 2 * L.tok_bytes;
     L.uf = o; o += kda ? rp * 512 : 0;
     L.gnv = o; o += kda ? 512 : 0;
+    L.xo = o; o += 512;
     L.am = o; o += round_up((4 * TC_NPAD * (TC_NPAD + 4) + 2 * TC_NPAD * rp + 6 * TC_NPAD + 4) * 4, 16);
     L.bars = o; o += 8 * (TC_NS + 5);
     L.slot = o; o += 16;
@@ -292,12 +294,13 @@ __device__ __forceinline__ float dot4(float4 a, float4 b) {
     return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, a.w * b.w)));
 }
 
-template <int KIND, int RP>
+template <int KIND, int RP, bool READ>
 __global__ void __launch_bounds__(TC_THREADS, 1)
 update_window_delta_tc(const __grid_constant__ CUtensorMap tmS, float *__restrict__ P,
                      const float *__restrict__ U, const __nv_bfloat16 *__restrict__ kbuf,
                      const __nv_bfloat16 *__restrict__ vbuf, const float *__restrict__ abuf,
-                     const float *__restrict__ bbuf, int B, int H, int r, int n, int W) {
+                     const float *__restrict__ bbuf, const __nv_bfloat16 *__restrict__ qv,
+                     float *__restrict__ o, int B, int H, int r, int n, int W) {
     using QT = __nv_bfloat16;
     constexpr bool KD = KIND == KDA;
     constexpr int NPAD = TC_NPAD, NK = tc_nk(KD), N1 = tc_n1(RP, KD), as = NPAD + 4;  // A, G rows: 16-B aligned
@@ -332,6 +335,7 @@ update_window_delta_tc(const __grid_constant__ CUtensorMap tmS, float *__restric
     const uint32_t b1_a = smem_u32(b1), kbm_a = smem_u32(kbm);
     float *uf = reinterpret_cast<float *>(sm + L.uf);    // KDA: [RP][128] basis rows of the current h
     float *gnv = reinterpret_cast<float *>(sm + L.gnv);  // KDA: [128] the window's decay product g_{n-1}
+    float *xo = reinterpret_cast<float *>(sm + L.xo);    // [128] the exact read, second column half
     const int kbytes = n * 128 * (int)sizeof(QT);
     constexpr int AOFF = 2 * NPAD * 128 * (int)sizeof(QT);  // KDA: decay rows after the keys and values
 
@@ -817,6 +821,8 @@ update_window_delta_tc(const __grid_constant__ CUtensorMap tmS, float *__restric
         tc_fence_after();
         // ---- step 5: S_n = g S_0 + D (KDA: g per key channel), back into the stage (its step-1 reads are
         // complete), then out by TMA tiled stores
+        float orow = 0.f;  // the exact read o = S_n^T q over this thread's 64 key channels
+        const QT *qh = READ ? qv + (size_t)head * 128 : nullptr;
 #pragma unroll
         for (int j2 = 0; j2 < 2; ++j2) {
             const int pnl = 2 * half + j2;
@@ -826,16 +832,23 @@ update_window_delta_tc(const __grid_constant__ CUtensorMap tmS, float *__restric
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 const float4 g4 = KD ? *reinterpret_cast<const float4 *>(gnv + 32 * pnl + 4 * q) : make_float4(g, g, g, g);
-                *reinterpret_cast<float4 *>(stage + pnl * TC_PANEL + sw128(row, 4 * q)) =
-                    make_float4(fmaf(g4.x, s0[32 * j2 + 4 * q], __uint_as_float(d[4 * q])),
-                                fmaf(g4.y, s0[32 * j2 + 4 * q + 1], __uint_as_float(d[4 * q + 1])),
-                                fmaf(g4.z, s0[32 * j2 + 4 * q + 2], __uint_as_float(d[4 * q + 2])),
-                                fmaf(g4.w, s0[32 * j2 + 4 * q + 3], __uint_as_float(d[4 * q + 3])));
+                const float4 sn = make_float4(fmaf(g4.x, s0[32 * j2 + 4 * q], __uint_as_float(d[4 * q])),
+                                              fmaf(g4.y, s0[32 * j2 + 4 * q + 1], __uint_as_float(d[4 * q + 1])),
+                                              fmaf(g4.z, s0[32 * j2 + 4 * q + 2], __uint_as_float(d[4 * q + 2])),
+                                              fmaf(g4.w, s0[32 * j2 + 4 * q + 3], __uint_as_float(d[4 * q + 3])));
+                *reinterpret_cast<float4 *>(stage + pnl * TC_PANEL + sw128(row, 4 * q)) = sn;
+                if constexpr (READ) {  // (the same query channels for every lane: broadcast loads)
+                    float qf[4];
+                    load4(qh + 32 * pnl + 4 * q, qf);
+                    orow = fmaf(sn.x, qf[0], fmaf(sn.y, qf[1], fmaf(sn.z, qf[2], fmaf(sn.w, qf[3], orow))));
+                }
             }
         }
+        if (READ && half == 1) xo[row] = orow;
         tc_fence_before();
         fence_proxy_async();  // the new state, written by these threads, is read by the TMA store
         __syncthreads();  // tensor memory and the operands are free for the next head
+        if (READ && half == 0) o[(size_t)head * 128 + row] = orow + xo[row];
         if (warp == 1) {
             if (elect_one()) {
                 for (int p = 0; p < 4; ++p) tma_store_2d(&tmS, 32 * p, head * 128, stage + p * TC_PANEL);
@@ -890,13 +903,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
 
 int update_tc_giveups(bool reset, unsigned *count) { return read_counter(&g_update_tc_giveups, reset, count); }
 
-// The delta-rule window update on the tensor cores, where it applies: Gated DeltaNet or KDA,
+// The delta-rule window update on the tensor cores, where it applies (with q and o: also the exact read
+// o = S_n^T q of the window's last step, from the updated fp32 state): Gated DeltaNet or KDA,
 // dk = dv = 128, fp32 state, bf16 keys and values (keys exact in TF32), 1 <= n <= 16 tokens,
 // r <= 16 (KDA: r <= 8, whose split decayed keys and basis rows take more shared memory).
 // Returns TC_NOT_APPLICABLE for other shapes (the caller then runs the CUDA-core kernel), else a
 // sketchssm_status.
 int launch_update_window_tc(const sketchssm_dims &d, void *S, float *P, const float *U, const void *k,
-                            const void *v, const float *alpha, const float *beta, int n, cudaStream_t stream) {
+                            const void *v, const float *alpha, const float *beta, int n, cudaStream_t stream,
+                            const void *q, float *o) {
     const bool kda = d.kind == SKSSM_KDA;
     if ((d.kind != SKSSM_GDN && !kda) || d.dk != 128 || d.dv != 128 || d.state_dtype != SKSSM_F32)
         return TC_NOT_APPLICABLE;
@@ -918,24 +933,37 @@ int launch_update_window_tc(const sketchssm_dims &d, void *S, float *P, const fl
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return SKSSM_ERR_CUDA;
 
-    auto run = [&](auto KINDc, auto RPc) -> int {
+    auto run = [&](auto KINDc, auto RPc, auto READc) -> int {
         constexpr int KIND = decltype(KINDc)::value, RP = decltype(RPc)::value;
-        auto kern = update_window_delta_tc<KIND, RP>;
+        auto kern = update_window_delta_tc<KIND, RP, decltype(READc)::value>;
         if (allow_max_smem(reinterpret_cast<const void *>(kern)) != SKSSM_OK) return SKSSM_ERR_CUDA;
         int sms = 0;
         if (sm_count(&sms) != SKSSM_OK) return SKSSM_ERR_CUDA;
         const int grid = NH < sms ? NH : sms;
         kern<<<grid, TC_THREADS, L.total, stream>>>(map, P, U, static_cast<const __nv_bfloat16 *>(k),
-                                                    static_cast<const __nv_bfloat16 *>(v), alpha, beta, d.B, d.H, d.r,
-                                                    n, d.W);
+                                                    static_cast<const __nv_bfloat16 *>(v), alpha, beta,
+                                                    static_cast<const __nv_bfloat16 *>(q), o, d.B, d.H, d.r, n, d.W);
         return launch_status();
     };
     using G = std::integral_constant<int, GDN>;
     using K = std::integral_constant<int, KDA>;
-    if (kda) return rp == 4 ? run(K(), std::integral_constant<int, 4>()) : run(K(), std::integral_constant<int, 8>());
-    if (rp == 4) return run(G(), std::integral_constant<int, 4>());
-    if (rp == 8) return run(G(), std::integral_constant<int, 8>());
-    return run(G(), std::integral_constant<int, 16>());
+    using R4 = std::integral_constant<int, 4>;
+    using R8 = std::integral_constant<int, 8>;
+    using R16 = std::integral_constant<int, 16>;
+    using NoRead = std::false_type;
+    if (kda) {  // (the fused read is taken for Gated DeltaNet only)
+        if (q != nullptr) return TC_NOT_APPLICABLE;
+        return rp == 4 ? run(K(), R4(), NoRead()) : run(K(), R8(), NoRead());
+    }
+    if (q != nullptr) {
+        using Read = std::true_type;
+        if (rp == 4) return run(G(), R4(), Read());
+        if (rp == 8) return run(G(), R8(), Read());
+        return run(G(), R16(), Read());
+    }
+    if (rp == 4) return run(G(), R4(), NoRead());
+    if (rp == 8) return run(G(), R8(), NoRead());
+    return run(G(), R16(), NoRead());
 }
 
 }  // namespace skssm

@@ -193,9 +193,9 @@ def test_config4_sweep_points(pt):
     _sampled(wl.workload(4, **pt), n_windows=1, n_heads=32)
 
 
-@pytest.mark.parametrize("cfg_id", [2, 3])
+@pytest.mark.parametrize("cfg_id", [1, 2, 3])
 def test_full_length_schedule(cfg_id):
-    """All 256 decode steps (16 windows) of the GDN and KDA workloads at full batch, on sampled
-    heads: error growth across every window of the run stays within the contract."""
+    """All 256 decode steps (16 windows) of the Mamba-2, GDN and KDA workloads at full batch, on
+    sampled heads: error growth across every window of the run stays within the contract."""
     cfg = wl.CONFIGS[cfg_id]
     _sampled(cfg, n_windows=cfg.steps // cfg.W, n_heads=24, label=f"{cfg.describe()} (all {cfg.steps} steps)")

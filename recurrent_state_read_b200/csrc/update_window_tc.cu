@@ -44,10 +44,11 @@
 // into the stage, from where it leaves by TMA tiled stores (a thread per row
 // storing to global memory directly costs one transaction per row per store).
 // The keys and values arrive by 1-D bulk copies one head ahead.  Roles: warp 0
-// issues the MMAs, warp 1 the copies; warps 2, 3, 6 and 7 compute the key Gram,
-// K U^T and the system matrix A[t][s] = b_t gamma_{t,s} (k_t . k_s) under step 1
-// (off the issuers' sub-partitions); warps 0-3 (one value channel per thread)
-// solve, while warp 4 builds the next head's decay products.  Tensor memory (512
+// issues the MMAs, warp 1 the copies; warps 2, 3, 6 and 7 compute the key Gram and
+// the system matrix A[t][s] = b_t gamma_{t,s} (k_t . k_s) under step 1 (off the
+// issuers' sub-partitions), warps 1 and 5 K U^T (r <= 8; for r = 16 the Gram
+// warps take it too); warps 0-3 (one value channel per thread) solve, while
+// warp 4 builds the next head's decay products.  Tensor memory (512
 // columns): the remainder (128), [X | S_0^T U] (<= 128), D (128), W~ hi | lo (32).
 // KDA (decay per key channel i, S_t = (I - b_t k_t k_t^T) diag(a_t) S_{t-1} + b_t k_t v_t^T): the
 // same steps with g_t, gamma_{t,s} per channel, x_t = S_0^T (g_t o k_t), A[t][s] = b_t
@@ -476,24 +477,48 @@ update_window_delta_tc(const __grid_constant__ CUtensorMap tmS, float *__restric
             const int tt = t0 + 2 * g + (lane >> 4), ss = lane & 15;
             Am[(buf * NPAD + tt) * as + ss] = Gam[(buf * NPAD + tt) * as + ss] * v[0];
         }
+        if constexpr (RP > 8) {  // K U^T (U = hi + lo) here too: 16 basis rows would make warps 1 and 5 the
+                                 // slower side (measured)
 #pragma unroll
-        for (int m0 = 0; m0 < RP; m0 += 8) {  // K U^T with U = hi + lo, eight basis rows at a time
-            float4 uu[8];
+            for (int m0 = 0; m0 < RP; m0 += 8) {
+                float4 uu[8];
 #pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                if (m0 + m < RP) {
+                for (int m = 0; m < 8; ++m) {
                     const float4 uh = rowv(NK + m0 + m), ul = rowv(NK + RP + m0 + m);
                     uu[m] = make_float4(uh.x + ul.x, uh.y + ul.y, uh.z + ul.z, uh.w + ul.w);
-                } else {
-                    uu[m] = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
-            }
-            float v[32];  // index i = 8 (row) + m
+                float v[32];  // index i = 8 (row) + m
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = dot4(kt[i >> 3], uu[i & 7]);
+                for (int i = 0; i < 32; ++i) v[i] = dot4(kt[i >> 3], uu[i & 7]);
+                warp_reduce_scatter32(v, lane);
+                kus[(buf * NPAD + t0 + (lane >> 3)) * RP + m0 + (lane & 7)] = v[0];
+            }
+        }
+    };
+    // GDN with RP <= 8, warps 1 and 5 (idle under step 1 once warp 1 has issued its copy): K U^T with U = hi + lo for
+    // key rows 8 (warp / 4) .. + 7, into buffer buf
+    auto ku_system = [&](int buf) {
+        const int t0 = 8 * (warp >> 2);
+        const unsigned char *pn = b1 + (lane >> 3) * B1P;
+        auto rowv = [&](int rr) {
+            return *reinterpret_cast<const float4 *>(pn + rr * 128 + ((((lane & 7) ^ rr) & 7) << 4));
+        };
+        float4 kt[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) kt[j] = rowv(t0 + j);
+#pragma unroll
+        for (int m0 = 0; m0 < RP; m0 += 4) {  // four basis rows at a time: 8 rows x 4 = 32 dots
+            float4 uu[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const float4 uh = rowv(NK + m0 + m), ul = rowv(NK + RP + m0 + m);
+                uu[m] = make_float4(uh.x + ul.x, uh.y + ul.y, uh.z + ul.z, uh.w + ul.w);
+            }
+            float v[32];  // index i = 4 (row) + m
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = dot4(kt[i >> 2], uu[i & 3]);
             warp_reduce_scatter32(v, lane);
-            const int m = m0 + (lane & 7);
-            if (m < RP) kus[(buf * NPAD + t0 + (lane >> 3)) * RP + m] = v[0];
+            kus[(buf * NPAD + t0 + (lane >> 2)) * RP + m0 + (lane & 3)] = v[0];
         }
     };
 
@@ -711,8 +736,10 @@ update_window_delta_tc(const __grid_constant__ CUtensorMap tmS, float *__restric
                 mma_commit(bar_1);
             }
             __syncwarp();
-        } else if ((warp & 2) != 0) {  // ---- step 2 under step 1
+        } else if ((warp & 2) != 0) {  // ---- step 2 under step 1: the Gram (and, for KDA, K U^T)
             gram_system(db, tk);
+        } else if (!KD && RP <= 8 && (warp == 1 || warp == 5)) {  // GDN's K U^T
+            ku_system(db);
         }
         // ---- step 1 complete
         if (warp == 0) ok = mbar_wait(bar_1, ph);

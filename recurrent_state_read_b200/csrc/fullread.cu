@@ -2,7 +2,7 @@
 // writes the whole state and returns o = S_t^T q_t.
 //
 // This is the access pattern the SketchSSM abstract compares against (the
-// "standard vLLM baseline"), and the one the agihunt digest's "Background"
+// standard vLLM decode path), and the one the agihunt digest's "Background"
 // bullet describes: every decode step reads the full recurrent state.  The
 // kernel streams each head's state once (one read, one write) with the same
 // register tile as the window update, and folds the read into the same pass:

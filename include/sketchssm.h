@@ -222,9 +222,9 @@ int sketchssm_update_window_seqs(const sketchssm_dims *dims, void *S, float *P, 
 
 /*
  * sketchssm_fullread_decode -- the baseline: one decode step with a full-state
- * read, as a standard serving engine does it (SketchSSM abstract, "standard
- * vLLM baseline"; digest bullet "Background": the full recurrent state is read
- * at every decode step).  Per head: S <- M S + b k v^T with this step's token,
+ * read, as a standard serving engine does it (SketchSSM abstract: the vLLM
+ * decode path it is compared with; digest bullet "Background": the full
+ * recurrent state is read at every decode step).  Per head: S <- M S + b k v^T with this step's token,
  * S stored back (state_dtype), o = S^T q from the updated fp32 values.
  *   S in/out [B][H][dv][dk];  q, k in [B][H][dk];  v in [B][H][dv];
  *   alpha in [B][H] (KDA [B][H][dk]);  beta in [B][H] (NULL for Mamba-2);

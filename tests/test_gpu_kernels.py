@@ -60,6 +60,7 @@ CASES = [
     ("kda", 128, 128, 128, 64, torch.float32, torch.float32),  # largest layout: one CTA per head
     ("gdn", 128, 128, 4, 24, torch.float32, torch.float32),    # fp32 tokens: the CUDA-core update
     ("gdn", 128, 128, 16, 13, torch.float32, torch.bfloat16),  # n = 13: the tensor-core update, r = 16
+    ("gdn", 128, 128, 8, 32, torch.float32, torch.bfloat16),   # W = 32: n = 16 on the tensor cores
 ]
 
 
